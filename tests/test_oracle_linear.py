@@ -1,0 +1,99 @@
+"""Pins of the oracle's GEMM reference and static-FP8 path: special cases that
+reduce to a plain matmul, checked against an exact triple loop, and the
+per-channel/per-tensor scale algebra on hand-sized inputs."""
+
+import numpy as np
+
+from oracle import formats as F
+from oracle import linear as L
+from oracle import quant as Q
+
+
+def _triple_loop(x, w, b):
+    M, K = x.shape
+    N = w.shape[0]
+    y = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += float(x[m, k]) * float(w[n, k])
+            y[m, n] = acc + (0.0 if b is None else float(b[n]))
+    return y
+
+
+def test_int4_unit_scales_reduce_to_plain_matmul():
+    # integer weights in [-7, 7] with every group holding a +-7: s = 1 exactly,
+    # so DQ(W) = W and y = x W^T + b
+    rng = np.random.default_rng(0)
+    w = rng.integers(-7, 8, (5, 256)).astype(np.float64)
+    w[:, ::128] = 7.0
+    x = rng.integers(-3, 4, (3, 256)).astype(np.float64) * 0.5
+    b = np.array([0.5, -1.0, 2.0, 0.0, 0.25])
+    st = L.quantize_pack("int4", w)
+    assert (F.bf16_from_bits(st["scales"]) == 1.0).all()
+    wd = L.dequant_exact("int4", st["packed"], st["scales"])
+    assert np.array_equal(wd, w)
+    assert np.array_equal(L.linear_ref(x, wd, b), _triple_loop(x, w, b))
+
+
+def test_mxfp4_zero_exponent_reduces_to_e2m1_matmul():
+    # every block max 6 -> e = 0: DQ(W) = W when W lies on the E2M1 grid
+    rng = np.random.default_rng(1)
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -.5, -1, -1.5, -2, -3, -4, -6])
+    w = rng.choice(grid, (4, 64))
+    w[:, ::32] = 6.0
+    x = rng.normal(size=(2, 64)).astype(np.float32).astype(np.float64)
+    st = L.quantize_pack("mxfp4", w)
+    assert (st["scales"] == 127).all()
+    wd = L.dequant_exact("mxfp4", st["packed"], st["scales"])
+    assert np.array_equal(wd, w)
+    np.testing.assert_allclose(L.linear_ref(x, wd), _triple_loop(x, w, None), rtol=0, atol=1e-12)
+
+
+def test_linear_ref_generic_matches_triple_loop():
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=(3, 32))
+    w = rng.normal(size=(4, 32))
+    b = rng.normal(size=4)
+    np.testing.assert_allclose(L.linear_ref(x, w, b), _triple_loop(x, w, b), rtol=1e-13, atol=1e-13)
+
+
+def test_static_linear_unit_scales_is_integer_matmul():
+    # with s_x = s_w = 1 and x, W on small E4M3 integers the layer is x W^T
+    rng = np.random.default_rng(3)
+    x = rng.integers(-8, 9, (2, 32)).astype(np.float64)
+    w = rng.integers(-8, 9, (3, 32)).astype(np.float64)
+    qx = L.quantize_act_fp8(x, 1.0)
+    qw = F.e4m3_encode(w)
+    y = L.static_linear(qx, 1.0, qw, np.ones(3))
+    assert np.array_equal(y, _triple_loop(x, w, None))
+
+
+def test_static_linear_scale_algebra():
+    # y scales linearly with s_x and with each channel's s_w
+    rng = np.random.default_rng(4)
+    qx = F.e4m3_encode(F.e4m3_round(rng.normal(0, 30, (2, 16))))
+    qw = F.e4m3_encode(F.e4m3_round(rng.normal(0, 30, (3, 16))))
+    base = L.static_linear(qx, 1.0, qw, np.ones(3))
+    y = L.static_linear(qx, 0.25, qw, np.array([1.0, 2.0, 0.5]))
+    assert np.array_equal(y, base * 0.25 * np.array([1.0, 2.0, 0.5])[None, :])
+
+
+def test_static_weight_scale_uses_symmetric_range():
+    w = np.array([[-3.0, 1.0, 2.0, 0.0] * 4, [0.5, -0.25, 0.125, 0.0] * 4])
+    codes, s = Q.quantize_fp8_rows(w)
+    assert s.tolist() == [float(F.f32(3.0 / 448)), float(F.f32(0.5 / 448))]
+
+
+def test_calibration_uses_min_max_over_all_batches():
+    w1 = np.eye(4)
+    batches = [np.array([[1.0, -2.0, 0.5, 0.0]]), np.array([[0.0, 3.5, -1.0, 0.0]])]
+    s1, s2 = L.calibrate_static_mlp(batches, w1, np.eye(4))
+    assert s1 == float(F.f32(3.5 / 448)) and s2 == float(F.f32(3.5 / 448))
+
+
+def test_sqnr_limits():
+    a = np.array([3.0, 4.0])
+    assert np.isclose(L.sqnr(a, a), 20 * np.log10(5.0 / 1e-12))
+    assert np.isclose(L.sqnr(a, np.zeros(2)), 0.0)
