@@ -1,0 +1,601 @@
+#!/usr/bin/env python
+"""Benchmark of the dequantize-in-prologue quantized Linear on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the pages' nn.Linear(3072, 4096) on x[32, 3072] in each weight-only format
+(INT4 g128, NVFP4, MXFP4, FP8 E4M3 per-channel) plus the static-FP8 page's
+two-layer 256->512->128 model on x[32, 256] -- six dqgemm_run calls.  The
+metric is microseconds per call (step time / 6), lower is better.
+
+Weights rotate round-robin over R independent weight sets whose packed bytes
+total at least 3x the L2 size, so every call streams its weight from HBM.
+The timed region is K steps replayed as CUDA graphs (one graph per weight
+set), bracketed by a barrier and a device synchronize, timed with CUDA
+events; multi-GPU runs are independent replicas (no data-path collective)
+and report the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep        # M x (K, N) x format sweep, one JSON line per point
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DQ-GEMM µs/call; HBM GB/s (M≤128) & TFLOP/s (M≥1024) vs B200 roofline"
+UNIT = "µs/call"
+LIN_FORMATS = ("int4", "nvfp4", "mxfp4", "fp8")
+LM, LK, LN = 32, 3072, 4096
+MLP_IN, MLP_HID, MLP_OUT = 256, 512, 128
+CALLS_PER_STEP = len(LIN_FORMATS) + 2
+WORKLOAD = ("Linear(3072->4096), x[32,3072] bf16, in INT4-g128 / NVFP4 / MXFP4 / FP8-WO + "
+            "static-FP8 MLP 256->512->128 (no bias), x[32,256]; 6 calls per step")
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+
+def algorithmic_bytes(fmt, M, K, N, bias=True):
+    """Bytes one call must move: packed weight + scales (+ global scale) + x + y + bias."""
+    if fmt == "int4":
+        w = N * K // 2 + N * (K // 128) * 2
+    elif fmt == "nvfp4":
+        w = N * K // 2 + N * (K // 16) + 4
+    elif fmt == "mxfp4":
+        w = N * K // 2 + N * (K // 32)
+    else:
+        w = N * K + N * 4
+    return w + M * K * 2 + M * N * 2 + (N * 2 if bias else 0)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_only_quantized_prologue_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def ncu_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("per_launch_bytes")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the GPU is busy."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"dq_clocks_{os.getpid()}_{gpu_index}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the workload on the GPU
+# ---------------------------------------------------------------------------
+
+
+class WeightSet:
+    """One independent set of every layer of the step, packed on the GPU."""
+
+    def __init__(self, idx, torch, dq, synthetic):
+        self.layers = {}
+        dev = "cuda"
+        for j, fmt in enumerate(LIN_FORMATS):
+            x, w, b = synthetic.linear_inputs(LM, LK, LN, seed=1000 * idx + j)
+            self.layers[fmt] = dq.QuantizedLinear.from_float(fmt, w.to(dev), b.to(dev))
+            if j == 0:
+                self.x = x.to(dev)
+        w1, w2 = synthetic.mlp_weights(seed=1000 * idx + 7)
+        w1, w2 = w1.to(dev), w2.to(dev)
+        # calibration: per-tensor min/max observers over ten seeded batches of
+        # the float bf16 model (static FP8 page, "Calibrate, then insert ...")
+        lo1 = hi1 = lo2 = hi2 = 0.0
+        for s in range(1, 11):
+            xc = synthetic.activations(LM, MLP_IN, seed=s).to(dev)
+            hc = xc @ w1.t()
+            lo1, hi1 = min(lo1, xc.min().item()), max(hi1, xc.max().item())
+            lo2, hi2 = min(lo2, hc.min().item()), max(hi2, hc.max().item())
+        s1 = float(torch.tensor(max(abs(lo1), abs(hi1)), dtype=torch.float32) / 448.0)
+        s2 = float(torch.tensor(max(abs(lo2), abs(hi2)), dtype=torch.float32) / 448.0)
+        self.mlp1 = dq.QuantizedLinear.from_float("fp8_static", w1.float(), None, act_scale=s1)
+        self.mlp2 = dq.QuantizedLinear.from_float("fp8_static", w2.float(), None, act_scale=s2)
+        self.xm = synthetic.activations(LM, MLP_IN, seed=1000 * idx + 8).to(dev)
+        self.y = {f: torch.empty((LM, LN), dtype=torch.bfloat16, device=dev) for f in LIN_FORMATS}
+        self.h = torch.empty((LM, MLP_HID), dtype=torch.bfloat16, device=dev)
+        self.ym = torch.empty((LM, MLP_OUT), dtype=torch.bfloat16, device=dev)
+        self.weight_bytes = sum(l.plan(LM)["weight_bytes"] for l in self.layers.values()) + \
+            self.mlp1.plan(LM)["weight_bytes"] + self.mlp2.plan(LM)["weight_bytes"]
+
+    def calls(self):
+        """(name, layer, x, y) in step order."""
+        out = [(f, self.layers[f], self.x, self.y[f]) for f in LIN_FORMATS]
+        out.append(("fp8_static_l1", self.mlp1, self.xm, self.h))
+        out.append(("fp8_static_l2", self.mlp2, self.h, self.ym))
+        return out
+
+    def step(self, torch, events=None):
+        for i, (name, layer, x, y) in enumerate(self.calls()):
+            if events is not None:
+                events[i][0].record()
+            layer(x, out=y)
+            if events is not None:
+                events[i][1].record()
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import weight_only_quantized_prologue_b200 as dq
+    from weight_only_quantized_prologue_b200 import synthetic
+
+    torch.cuda.set_device(local_rank)
+    props = torch.cuda.get_device_properties(local_rank)
+    l2 = getattr(props, "L2_cache_size", 126 * 2**20)
+    first = WeightSet(0, torch, dq, synthetic)
+    R = max(2, math.ceil(3 * l2 / first.weight_bytes))
+    sets = [first] + [WeightSet(i, torch, dq, synthetic) for i in range(1, R)]
+    for s in sets:                       # first calls allocate split-K workspaces
+        s.step(torch)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    graphs = []
+    with torch.cuda.stream(stream):
+        for s in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                s.step(torch)
+            graphs.append(g)
+        # a second graph family with CUDA events around every call, for the
+        # per-kernel durations behind the roofline figure
+        n_ev = 2 * R
+        ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(CALLS_PER_STEP)]
+              for _ in range(n_ev)]
+        g_ev = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_ev, stream=stream):
+            for i in range(n_ev):
+                sets[i % R].step(torch, events=ev[i])
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    with torch.cuda.stream(stream):
+        if sampler:
+            sampler.start()
+        settle_until = time.time() + 1.5          # clocks settle under load (untimed)
+        i = 0
+        while time.time() < settle_until:
+            graphs[i % R].replay()
+            i += 1
+            if i % 200 == 0:
+                stream.synchronize()
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+        stream.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            graphs[i % R].replay()
+        t1.record(stream)
+        t1.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+        ms_local = t0.elapsed_time(t1)
+        clocks = sampler.stop() if sampler else None
+
+        # per-kernel durations (events inside the graph)
+        g_ev.replay()
+        torch.cuda.synchronize()
+    names = [c[0] for c in first.calls()]
+    per_call = {n: statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(n_ev)) * 1000.0
+                for j, n in enumerate(names)}
+
+    ms = ms_local
+    if world > 1:
+        ms = aggregate_max(ms_local)
+
+    # end-to-end through the public API with host buffers: per call, pinned
+    # host x -> device, dqgemm_run, device y -> pinned host
+    e2e_steps = max(3, min(args.steps, 200))
+    host = []
+    for s in sets:
+        hx = {n: x.cpu().pin_memory() for (n, _, x, _) in s.calls() if n != "fp8_static_l2"}
+        hy = {n: y.cpu().pin_memory() for (n, _, _, y) in s.calls() if n != "fp8_static_l1"}
+        host.append((hx, hy))
+    h2d = sum(x.numel() * 2 for (n, _, x, _) in first.calls() if n != "fp8_static_l2")
+    d2h = sum(y.numel() * 2 for (n, _, _, y) in first.calls() if n != "fp8_static_l1")
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            _e2e_step(sets[i % R], host[i % R])
+        stream.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            _e2e_step(sets[i % R], host[i % R])
+        e1.record(stream)
+        e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        e2e_ms = aggregate_max(e2e_ms)
+
+    for s in sets:
+        for l in list(s.layers.values()) + [s.mlp1, s.mlp2]:
+            assert l.last_error() == 0, "device-side wait timed out"
+
+    value = ms * 1000.0 / (args.steps * CALLS_PER_STEP * world)
+    peaks = measured_peaks()
+    lin = {n: per_call[n] for n in LIN_FORMATS}
+    dom = max(lin, key=lin.get)
+    alg = algorithmic_bytes(dom, LM, LK, LN)
+    achieved = alg / (lin[dom] * 1e-6) / 1e9
+    traffic = ncu_traffic()
+    roofline = {"bound": "hbm", "kernel": f"dq_gemm_kernel<{dom}, BN=32>", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": (traffic or {}).get(dom), "algorithmic_bytes": alg,
+                "avg_launch_us": round(lin[dom], 3), "peak_source": f"{peaks['source']} (HBM copy)"}
+    per_format = {n: {"us": round(per_call[n], 3),
+                      "GB/s": round(algorithmic_bytes(n, LM, LK, LN) / (per_call[n] * 1e-6) / 1e9, 1),
+                      "frac_hbm": round(algorithmic_bytes(n, LM, LK, LN) / (per_call[n] * 1e-6) / 1e9
+                                        / peaks["hbm_gbs"], 4)} for n in LIN_FORMATS}
+    per_format["fp8_static_l1"] = {"us": round(per_call["fp8_static_l1"], 3)}
+    per_format["fp8_static_l2"] = {"us": round(per_call["fp8_static_l2"], 3)}
+    result = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": LM, "K": LK, "N": LN, "formats": list(LIN_FORMATS) + ["fp8_static"],
+                   "weight_sets": R, "rotated_weight_MB": round(R * first.weight_bytes / 2**20, 1),
+                   "l2_defeat": f"weights rotate over {R} sets >= 3x L2 ({l2 // 2**20} MB)",
+                   "parallelism": f"replicas x{world}", "timing": "CUDA graphs, CUDA events"},
+        "per_call": per_format,
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_ms * 1000.0 / (e2e_steps * CALLS_PER_STEP * world), 4), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * CALLS_PER_STEP,
+        "clocks": clocks,
+    }
+    return result, sets
+
+
+def _e2e_step(s, host):
+    hx, hy = host
+    calls = s.calls()
+    for name, layer, x, y in calls:
+        if name in hx:
+            x.copy_(hx[name], non_blocking=True)
+        layer(x, out=y)
+        if name in hy:
+            hy[name].copy_(y, non_blocking=True)
+
+
+def aggregate_max(v):
+    """Max of a per-rank float over all ranks (the contract's device-time max)."""
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+
+class OracleWorkload:
+    """The same step computed by the fp64 oracle from its own packed storage
+    (quantization itself is not timed: the GPU path also packs once)."""
+
+    def __init__(self, synthetic):
+        import numpy as np
+
+        from oracle import linear as L
+
+        self.L, self.np = L, np
+        x, w, b = synthetic.linear_inputs(LM, LK, LN, seed=0)
+        self.x = x.float().numpy().astype(np.float64)
+        self.b = b.float().numpy().astype(np.float64)
+        self.store = {f: L.quantize_pack(f, w.numpy().astype(np.float64)) for f in LIN_FORMATS}
+        w1, w2 = synthetic.mlp_weights(seed=7)
+        w1v, w2v = w1.float().numpy().astype(np.float64), w2.float().numpy().astype(np.float64)
+        cal = [synthetic.activations(LM, MLP_IN, seed=s).float().numpy().astype(np.float64) for s in range(1, 11)]
+        self.s1, self.s2 = L.calibrate_static_mlp(cal, w1v, w2v)
+        self.q1 = L.quantize_pack("fp8", w1v)
+        self.q2 = L.quantize_pack("fp8", w2v)
+        self.xm = synthetic.activations(LM, MLP_IN, seed=8).float().numpy().astype(np.float64)
+        from oracle.formats import bf16
+        self.h = bf16(L.static_linear(L.quantize_act_fp8(self.xm, self.s1), self.s1,
+                                      self.q1["packed"], self.q1["scales"]))
+
+    def call(self, name, rows=None):
+        """One call of the step; `rows` restricts the weight to its first
+        `rows` output channels (a bounded sample of the call)."""
+        L = self.L
+        if name in LIN_FORMATS:
+            st = self.store[name]
+            p, s = st["packed"], st["scales"]
+            if rows is not None:
+                p, s = p[:rows], s[:rows]
+            wd = L.dequant_exact(name, p, s, st["global_scale"])
+            return L.linear_ref(self.x, wd, self.b[: wd.shape[0]])
+        if name == "fp8_static_l1":
+            p, s = self.q1["packed"], self.q1["scales"]
+            return L.static_linear(L.quantize_act_fp8(self.xm, self.s1), self.s1, p[:rows], s[:rows])
+        p, s = self.q2["packed"], self.q2["scales"]
+        return L.static_linear(L.quantize_act_fp8(self.h, self.s2), self.s2, p[:rows], s[:rows])
+
+    def rows_of(self, name):
+        return {"fp8_static_l1": MLP_HID, "fp8_static_l2": MLP_OUT}.get(name, LN)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def time_oracle_step(ow, fraction):
+    """Seconds for one step of the oracle on `fraction` of each call's output
+    channels, and the seconds scaled to the full step."""
+    names = list(LIN_FORMATS) + ["fp8_static_l1", "fp8_static_l2"]
+    t = 0.0
+    for n in names:
+        rows = max(16, int(ow.rows_of(n) * fraction) // 16 * 16)
+        t0 = time.perf_counter()
+        ow.call(n, rows=rows)
+        t += (time.perf_counter() - t0) * ow.rows_of(n) / rows
+    return t
+
+
+def cpu_baseline(synthetic, budget_s=15.0):
+    ow = OracleWorkload(synthetic)
+    time_oracle_step(ow, 1.0 / 64)      # warm caches / BLAS
+    t_full, n = 0.0, 0
+    t_start = time.perf_counter()
+    while n < 2 or time.perf_counter() - t_start < budget_s:
+        t_full += time_oracle_step(ow, 1.0)
+        n += 1
+        if time.perf_counter() - t_start > 2 * budget_s:
+            break
+    us_per_call = t_full / n * 1e6 / CALLS_PER_STEP
+    return {"value": round(us_per_call, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} full oracle steps (6 calls each: dequantize-exact + fp64 GEMM, "
+                      f"storage packed beforehand), {time.perf_counter() - t_start:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    from weight_only_quantized_prologue_b200 import synthetic
+
+    if rank != 0:
+        return None
+    ow = OracleWorkload(synthetic)
+    # size each step so that warmup + steps end within ~2 minutes
+    probe = time_oracle_step(ow, 1.0 / 64)
+    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    fraction = min(1.0, max(1.0 / 256, per_step_budget / max(probe, 1e-9)))
+    for _ in range(args.warmup):
+        time_oracle_step(ow, fraction)
+    t0 = time.perf_counter()
+    scaled = 0.0
+    for _ in range(args.steps):
+        scaled += time_oracle_step(ow, fraction)
+    wall = time.perf_counter() - t0
+    value = scaled * 1e6 / (args.steps * CALLS_PER_STEP)
+    sample = (f"each step computes {fraction:.4g} of every call's output channels with the fp64 oracle "
+              f"(dequantize-exact + GEMM) and scales its time to the full call; {wall:.1f} s total")
+    return {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(scaled * 1000.0 / args.steps, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD, "M": LM, "K": LK, "N": LN,
+                       "formats": list(LIN_FORMATS) + ["fp8_static"], "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+# sweep (M x (K, N) x format), one JSON line per point
+# ---------------------------------------------------------------------------
+
+
+def run_sweep(args):
+    import torch
+
+    import weight_only_quantized_prologue_b200 as dq
+    from weight_only_quantized_prologue_b200 import synthetic
+
+    torch.cuda.set_device(0)
+    peaks = measured_peaks()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    Ms = [int(m) for m in args.sweep_m.split(",")]
+    shapes = [tuple(int(v) for v in s.split("x")) for s in args.sweep_kn.split(",")]
+    fmts = args.sweep_formats.split(",")
+    for (K, N) in shapes:
+        for fmt in fmts:
+            wb = algorithmic_bytes("fp8" if fmt == "fp8_static" else fmt, 0, K, N, bias=False)
+            R = max(2, math.ceil(3 * l2 / wb))
+            layers = []
+            for r in range(R):
+                _, w, b = synthetic.linear_inputs(1, K, N, seed=r)
+                layers.append(dq.QuantizedLinear.from_float(fmt, w.cuda(), None if fmt == "fp8_static" else b.cuda(),
+                                                            act_scale=0.02))
+            for M in Ms:
+                x = synthetic.activations(M, K, seed=1).cuda()
+                y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+                for l in layers:
+                    l(x, out=y)
+                torch.cuda.synchronize()
+                flops = 2.0 * M * K * N
+                reps = max(R, min(400, int(2e11 / max(flops, 1))))
+                stream = torch.cuda.Stream()
+                with torch.cuda.stream(stream):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        for i in range(reps):
+                            layers[i % R](x, out=y)
+                    g.replay()
+                    stream.synchronize()
+                    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    t0.record(stream)
+                    g.replay()
+                    t1.record(stream)
+                    t1.synchronize()
+                us = t0.elapsed_time(t1) * 1000.0 / reps
+                byts = algorithmic_bytes("fp8" if fmt == "fp8_static" else fmt, M, K, N,
+                                         bias=fmt != "fp8_static")
+                gbs = byts / (us * 1e-6) / 1e9
+                tflops = flops / (us * 1e-6) / 1e12
+                peak_t = peaks["bf16_tflops"] * (2.0 if fmt == "fp8_static" else 1.0)
+                print(json.dumps({"fmt": fmt, "M": M, "K": K, "N": N, "us": round(us, 3),
+                                  "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                  "TFLOP/s": round(tflops, 1), "frac_tensor": round(tflops / peak_t, 4),
+                                  "plan": layers[0].plan(M)}), flush=True)
+                del g
+            for l in layers:
+                l.close()
+
+
+# ---------------------------------------------------------------------------
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--sweep-m", default="1,16,32,128,1024,4096")
+    ap.add_argument("--sweep-kn", default="4096x4096,4096x14336,14336x4096")
+    ap.add_argument("--sweep-formats", default="int4,nvfp4,mxfp4,fp8,fp8_static")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.sweep:
+        run_sweep(args)
+        return
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    res, sets = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            from weight_only_quantized_prologue_b200 import synthetic
+            res["cpu_baseline"] = cpu_baseline(synthetic)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * dqgemm.h -- C ABI of libdqgemm: a quantized nn.Linear for NVIDIA B200
+ * (sm_100a) whose low-bit weight stays packed in HBM and is dequantized in
+ * the prologue of a tcgen05 tensor-core GEMM:
+ *
+ *     y[M, N] = x[M, K] . deq(W)[N, K]^T + b[N]        (x, y, b in bf16)
+ *
+ * The operation is the one the Torch-TensorRT / TorchAO tutorial pages build
+ * as "weight constant + DQ prologue into GEMM":
+ *   - "TorchAO INT4 Weight-Only Quantization (Linear)", intro: symmetric
+ *     group-wise INT4 (zero-point 0, group_size=128), DQ prologue into GEMM.
+ *   - "TorchAO NVFP4 Weight-Only Quantization (Linear)", intro: packed FP4
+ *     E2M1 weights, FP8 E4M3 block scales, FP32 global scale, two-level DQ
+ *     prologue into a high-precision GEMM; activations stay bf16.
+ *   - "TorchAO MXFP4 Dynamic Activation + MX Weight (Linear)", intro: packed
+ *     E2M1 weights, E8M0 block scales, block size 32, weight DQ prologue.
+ *   - "TorchAO FP8 Weight-Only Quantization (Linear)", intro: FP8 weight
+ *     constant plus a DQ prologue fused into the matmul on Blackwell.
+ *   - "TorchAO Static FP8 Quantization (Linear)", intro and "Graph after
+ *     export": activations quantized to e4m3 with a calibrated per-tensor
+ *     scale, weights e4m3 per channel, GEMM in FP8 on the tensor cores.
+ *
+ * Conventions for every entry point
+ *   - All pointers are plain pointers.  "device" means memory the CUDA device
+ *     can address (cudaMalloc / torch CUDA tensors); "host" means CPU memory.
+ *   - Matrices are row-major and densely packed.  W is [N, K] as in
+ *     nn.Linear (out_features x in_features); groups / blocks run along K.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls that take a stream are asynchronous on it.
+ *   - Every entry point returns a dqgemm_status.  Argument checks are
+ *     synchronous.  Nothing aborts, throws or traps across this boundary.
+ *   - Device pointers must be 16-byte aligned (DQ_ERR_ALIGNMENT otherwise).
+ *   - The library never frees or retains caller memory.
+ */
+#ifndef DQGEMM_H
+#define DQGEMM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Weight formats and the canonical storage each takes at dqgemm_create.
+ *   DQ_INT4_G128   packed  u8 [N, K/2]: two's-complement nibbles, low nibble = even k
+ *                  scales  bf16 [N, K/128] (one per group of 128 along K)
+ *                  K % 128 == 0
+ *   DQ_NVFP4       packed  u8 [N, K/2]: E2M1 nibbles, low nibble = even k
+ *                  scales  u8 [N, K/16]: E4M3 block scales (one per 16 along K)
+ *                  global_scale: the FP32 global scale g;  K % 16 == 0, N % 16 == 0
+ *   DQ_MXFP4       packed  u8 [N, K/2]: E2M1 nibbles, low nibble = even k
+ *                  scales  u8 [N, K/32]: E8M0 block exponents 2^(e-127)
+ *                  K % 32 == 0, N % 32 == 0
+ *   DQ_FP8_WO      packed  u8 [N, K]: E4M3 codes;  scales fp32 [N] per channel
+ *                  K % 16 == 0
+ *   DQ_FP8_STATIC  as DQ_FP8_WO, plus global_scale = the calibrated fp32
+ *                  per-tensor activation scale s_x; the GEMM runs FP8 x FP8
+ *                  on e4m3(x / s_x) and rescales by s_x * s_w[n].
+ */
+typedef enum {
+  DQ_INT4_G128 = 0,
+  DQ_NVFP4 = 1,
+  DQ_MXFP4 = 2,
+  DQ_FP8_WO = 3,
+  DQ_FP8_STATIC = 4
+} dqgemm_format;
+
+typedef enum {
+  DQ_OK = 0,
+  DQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size or divisibility, unknown format */
+  DQ_ERR_UNSUPPORTED = 2,  /* valid request this build cannot serve (e.g. scale range) */
+  DQ_ERR_ALIGNMENT = 3,    /* a device pointer is not 16-byte aligned */
+  DQ_ERR_ALLOC = 4,        /* device or host allocation failed */
+  DQ_ERR_CUDA = 5,         /* a CUDA runtime/driver call or a launch failed */
+  DQ_ERR_TIMEOUT = 6       /* a bounded device-side wait expired (see dqgemm_last_error) */
+} dqgemm_status;
+
+typedef struct dqgemm_s* dqgemm_handle;
+
+/* Create a quantized Linear.  Reads `packed_w`, `scales` and `bias` (device
+ * pointers in the canonical layout above; `bias` is bf16 [N] or NULL), copies
+ * them, and re-lays the weight out into the kernel's tile order in device
+ * memory owned by the handle (the analogue of the INT4 page's "re-packs ...
+ * into an INT4 constant at build time", "Export and compile").  The caller may
+ * free its buffers afterwards; the weights are immutable for the handle's
+ * life.  Synchronizes the device.  On error *out is set to NULL. */
+dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt, int K, int N,
+                            const void* packed_w, const void* scales,
+                            float global_scale, const void* bias);
+
+/* y = x . deq(W)^T + b.  x: device bf16 [M, K]; y: device bf16 [M, N]; M >= 1.
+ * One kernel launch on `stream`.  For DQ_FP8_STATIC the activation is
+ * quantized to e4m3 inside the same kernel.  The handle owns a split-K
+ * workspace that grows on the first call with a larger M (that call
+ * allocates and synchronizes); calls on one handle must not overlap on
+ * different streams.  Device-side wait timeouts are reported through
+ * dqgemm_last_error after the stream has been synchronized. */
+dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream);
+
+/* Release the handle and its device memory (synchronizes the device). */
+dqgemm_status dqgemm_destroy(dqgemm_handle h);
+
+/* Debug: write the dequantized weight as bf16 [N, K] (device) from the
+ * handle's re-laid-out storage, through the same unpack code the GEMM
+ * prologue uses:  INT4 bf16(c*s);  NVFP4 bf16(f32(e2m1*dec(sb)*g));
+ * MXFP4 bf16(e2m1*2^(e-127));  FP8 bf16(f32(e4m3*s[n])).  -0.0 is kept. */
+dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream);
+
+/* Static-FP8 activation quantization (the Q node of the static FP8 page's
+ * "Graph after export"): q[m,k] = e4m3(f32(x[m,k] / s_x)), IEEE division,
+ * round to nearest even, saturating to +-448.  x: device bf16 [M, K];
+ * q: device u8 [M, K]; s_x > 0. */
+dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x,
+                                      void* q, void* stream);
+
+/* Quantize and pack a host fp32 weight [N, K] into the canonical layout of
+ * `fmt` (host outputs `packed` and `scales`, sized as listed above).  The
+ * recipes (fp32 operations, round to nearest even):
+ *   INT4   s = bf16(amax_group/7); c = clamp(rne(W/s), -8, 7); s == 0 -> c = 0
+ *   NVFP4  g = amax/2688 (1 if amax == 0); sb = e4m3((amax_blk16/6)/g);
+ *          c = e2m1(W/(dec(sb)*g)), saturating; 0 where the divisor is 0
+ *   MXFP4  e = floor(log2 amax_blk32) - 2 in [-127,127]; code e+127 (0 for a
+ *          zero block); c = e2m1(W * 2^-e), saturating
+ *   FP8    s[n] = max|W[n,:]|/448; c = e4m3(W/s[n]) (0 for a zero row)
+ * `global_scale` (host, may be NULL) receives g for NVFP4 and 1 otherwise.
+ * DQ_ERR_INVALID_ARG if W holds a non-finite value. */
+dqgemm_status dqgemm_pack_host(dqgemm_format fmt, const float* W, int K, int N,
+                               void* packed, void* scales, float* global_scale);
+
+/* Same as dqgemm_pack_host on the GPU: W, packed and scales are device
+ * pointers; results are bit-identical to dqgemm_pack_host.  If
+ * `global_scale` (host pointer) is not NULL the call synchronizes `stream`
+ * and stores g there.  Allocates and frees 4 bytes of device memory. */
+dqgemm_status dqgemm_pack_device(dqgemm_format fmt, const float* W, int K, int N,
+                                 void* packed, void* scales, float* global_scale,
+                                 void* stream);
+
+/* Status of the last device-side check of the handle's kernels (DQ_OK or
+ * DQ_ERR_TIMEOUT), then clears it.  Synchronizes the device. */
+dqgemm_status dqgemm_last_error(dqgemm_handle h);
+
+/* Diagnostic: launch a kernel whose only wait can never complete and which
+ * must give up after `timeout_us` microseconds; returns DQ_ERR_TIMEOUT when
+ * the bounded wait worked (the context stays usable), DQ_OK never.
+ * Synchronizes `stream`. */
+dqgemm_status dqgemm_selftest_timeout(int timeout_us, void* stream);
+
+/* Launch plan that dqgemm_run uses for a given M (for benchmarks and tests). */
+typedef struct {
+  int bn;               /* MMA N (activation rows per tile): 16, 32, 64 or 128 */
+  int m_tiles;          /* ceil(M / bn) */
+  int n_tiles;          /* ceil(N / 128) */
+  int k_stages;         /* ceil(K / 128) */
+  int grid;             /* CTAs launched (<= number of SMs) */
+  int max_segments;     /* most CTAs sharing one output tile (split-K depth) */
+  int stages;           /* shared-memory pipeline depth */
+  int smem_bytes;       /* dynamic shared memory per CTA */
+  long long workspace_bytes; /* split-K partial buffer the plan needs */
+  long long weight_bytes;    /* packed weight + scale bytes streamed per call */
+} dqgemm_plan;
+
+dqgemm_status dqgemm_get_plan(dqgemm_handle h, int M, dqgemm_plan* plan);
+
+/* Human-readable name of a status code (static storage). */
+const char* dqgemm_status_string(dqgemm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQGEMM_H */

@@ -1,0 +1,574 @@
+// dq_api.cu -- the C ABI declared in include/dqgemm.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "dq_aux.cuh"
+#include "dq_codec.h"
+#include "dq_gemm.cuh"
+#include "dqgemm.h"
+
+using namespace dq;
+
+struct dqgemm_s {
+  int fmt = 0, K = 0, N = 0;
+  int k_stages = 0, n_tiles = 0;
+  int device = 0, num_sms = 0;
+  uint8_t* wchunks = nullptr;       // pre-tiled weight
+  size_t wchunk_bytes = 0;
+  float* col_scale = nullptr;       // [N] for FP8 formats
+  __nv_bfloat16* bias = nullptr;    // [N] or null
+  int* status = nullptr;            // device status word
+  float sigma = 1.f, s_x = 1.f;
+  int mx_bias = 126;
+  float* ws = nullptr;              // split-K partials
+  size_t ws_bytes = 0;
+  int* counters = nullptr;          // per-tile arrival counters
+  size_t counters_n = 0;
+  long long weight_bytes = 0;       // canonical packed + scale bytes
+};
+
+namespace {
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;   // 2 s
+
+unsigned long long timeout_ns() {
+  static unsigned long long t = [] {
+    const char* e = std::getenv("DQGEMM_TIMEOUT_MS");
+    return e ? (unsigned long long)std::strtoull(e, nullptr, 10) * 1000000ull : kDefaultTimeoutNs;
+  }();
+  return t;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+// canonical storage sizes of dqgemm.h
+size_t packed_bytes(int fmt, int K, int N) { return is_4bit(fmt) ? (size_t)N * K / 2 : (size_t)N * K; }
+size_t scale_bytes(int fmt, int K, int N) {
+  switch (fmt) {
+    case FMT_INT4: return (size_t)N * (K / 128) * 2;
+    case FMT_NVFP4: return (size_t)N * (K / 16);
+    case FMT_MXFP4: return (size_t)N * (K / 32);
+    default: return (size_t)N * 4;
+  }
+}
+
+dqgemm_status check_shape(int fmt, int K, int N) {
+  if (fmt < 0 || fmt > 4 || K <= 0 || N <= 0) return DQ_ERR_INVALID_ARG;
+  switch (fmt) {
+    case FMT_INT4: return K % 128 ? DQ_ERR_INVALID_ARG : DQ_OK;
+    case FMT_NVFP4: return (K % 16 || N % 16) ? DQ_ERR_INVALID_ARG : DQ_OK;
+    case FMT_MXFP4: return (K % 32 || N % 32) ? DQ_ERR_INVALID_ARG : DQ_OK;
+    default: return K % 16 ? DQ_ERR_INVALID_ARG : DQ_OK;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host re-layout: canonical -> kernel tile order (see dq_layout.h)
+// ---------------------------------------------------------------------------
+void relayout(int fmt, int K, int N, int KS, int NT, const std::vector<uint8_t>& packed,
+              const std::vector<uint8_t>& scales, std::vector<uint8_t>& out) {
+  const int CH = chunk_bytes(fmt);
+  out.assign((size_t)NT * KS * CH, 0);
+  auto nib = [&](int n, int k) -> uint32_t {
+    if (n >= N || k >= K) return 0;
+    return (packed[(size_t)n * (K / 2) + k / 2] >> ((k & 1) * 4)) & 0xFu;
+  };
+  auto code8 = [&](int n, int k) -> uint32_t {
+    if (n >= N || k >= K) return 0;
+    return packed[(size_t)n * K + k];
+  };
+  auto put32 = [](uint8_t* p, uint32_t v) { std::memcpy(p, &v, 4); };
+  for (int t = 0; t < NT; ++t) {
+    for (int s = 0; s < KS; ++s) {
+      uint8_t* ch = out.data() + ((size_t)t * KS + s) * CH;
+      for (int r = 0; r < TILE_N; ++r) {
+        const int n = t * TILE_N + r;
+        if (is_4bit(fmt)) {
+          for (int h = 0; h < 2; ++h)
+            for (int j = 0; j < 2; ++j)
+              for (int w = 0; w < 4; ++w) {
+                const int k0 = s * STAGE_K + 64 * h + 32 * j + 8 * w;
+                uint32_t c[8], word = 0;
+                for (int i = 0; i < 8; ++i) c[i] = nib(n, k0 + i);
+                if (fmt == FMT_INT4) {
+                  for (int jj = 0; jj < 4; ++jj) word |= (c[2 * jj] << (4 * jj)) | (c[2 * jj + 1] << (16 + 4 * jj));
+                } else {
+                  uint32_t m[8], sg[8];
+                  for (int i = 0; i < 8; ++i) { m[i] = c[i] & 7u; sg[i] = c[i] >> 3; }
+                  word = m[0] | (m[1] << 16) | (sg[0] << 14) | (sg[1] << 30) |
+                         (m[2] << 3) | (m[3] << 19) | (sg[2] << 12) | (sg[3] << 28) |
+                         (m[4] << 6) | (m[5] << 22) | (sg[4] << 15) | (sg[5] << 31) |
+                         (m[6] << 9) | (m[7] << 25) | (sg[6] << 13) | (sg[7] << 29);
+                }
+                put32(ch + ((h * 2 + j) * TILE_N + r) * 16 + w * 4, word);
+              }
+          uint8_t* sc = ch + PACKED4_BYTES;
+          if (fmt == FMT_INT4) {
+            const int groups = K / 128;
+            uint16_t v = 0;
+            if (n < N && s < groups) std::memcpy(&v, &scales[((size_t)n * groups + s) * 2], 2);
+            std::memcpy(sc + r * 2, &v, 2);
+          } else if (fmt == FMT_NVFP4) {
+            const int blocks = K / 16;
+            for (int h = 0; h < 2; ++h)
+              for (int b = 0; b < 4; ++b) {
+                const int blk = s * 8 + 4 * h + b;
+                sc[(h * TILE_N + r) * 4 + b] = (n < N && blk < blocks) ? scales[(size_t)n * blocks + blk] : 0;
+              }
+          } else {
+            const int blocks = K / 32;
+            for (int h = 0; h < 2; ++h)
+              for (int b = 0; b < 2; ++b) {
+                const int blk = s * 4 + 2 * h + b;
+                sc[(h * TILE_N + r) * 2 + b] = (n < N && blk < blocks) ? scales[(size_t)n * blocks + blk] : 0;
+              }
+          }
+        } else if (fmt == FMT_FP8) {
+          for (int h = 0; h < 2; ++h)
+            for (int j = 0; j < 4; ++j)
+              for (int w = 0; w < 4; ++w) {
+                const int k0 = s * STAGE_K + 64 * h + 16 * j + 4 * w;
+                uint32_t b[4], m[4], sg[4];
+                for (int i = 0; i < 4; ++i) { b[i] = code8(n, k0 + i); m[i] = b[i] & 0x7Fu; sg[i] = b[i] >> 7; }
+                const uint32_t word = m[0] | (m[1] << 16) | (sg[0] << 15) | (sg[1] << 31) |
+                                      (m[2] << 7) | (m[3] << 23) | (sg[2] << 14) | (sg[3] << 30);
+                put32(ch + ((h * 4 + j) * TILE_N + r) * 16 + w * 4, word);
+              }
+        } else {  // static FP8: swizzled K-major shared-memory image
+          for (int kl = 0; kl < STAGE_K; ++kl)
+            ch[r * 128 + (((kl >> 4) ^ (r & 7)) << 4) + (kl & 15)] = (uint8_t)code8(n, s * STAGE_K + kl);
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tensor map for the bf16 activation x [M, K]: boxes of 64 k x BN rows, 128B swizzle
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+bool make_x_map(CUtensorMap* map, const void* x, int M, int K, int bn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)bn};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// launch dispatch
+// ---------------------------------------------------------------------------
+template <int FMT, int BN>
+struct GemmLauncher {
+  using C = GemmCfg<FMT, BN>;
+  static cudaError_t set_attr() {
+    return cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  }
+  static cudaError_t launch(const CUtensorMap& tm, const GemmParams& p, int grid, cudaStream_t st) {
+    dq_gemm_kernel<FMT, BN><<<grid, C::THREADS, C::SMEM, st>>>(tm, p);
+    return cudaGetLastError();
+  }
+};
+
+template <int FMT>
+int stages_for(int bn) {
+  switch (bn) {
+    case 16: return GemmCfg<FMT, 16>::STAGES;
+    case 32: return GemmCfg<FMT, 32>::STAGES;
+    case 64: return GemmCfg<FMT, 64>::STAGES;
+    default: return GemmCfg<FMT, 128>::STAGES;
+  }
+}
+template <int FMT>
+int smem_for(int bn) {
+  switch (bn) {
+    case 16: return GemmCfg<FMT, 16>::SMEM;
+    case 32: return GemmCfg<FMT, 32>::SMEM;
+    case 64: return GemmCfg<FMT, 64>::SMEM;
+    default: return GemmCfg<FMT, 128>::SMEM;
+  }
+}
+template <int FMT>
+cudaError_t set_attrs() {
+  cudaError_t e = GemmLauncher<FMT, 16>::set_attr();
+  if (e == cudaSuccess) e = GemmLauncher<FMT, 32>::set_attr();
+  if (e == cudaSuccess) e = GemmLauncher<FMT, 64>::set_attr();
+  if (e == cudaSuccess) e = GemmLauncher<FMT, 128>::set_attr();
+  return e;
+}
+template <int FMT>
+cudaError_t launch_fmt(int bn, const CUtensorMap& tm, const GemmParams& p, int grid, cudaStream_t st) {
+  switch (bn) {
+    case 16: return GemmLauncher<FMT, 16>::launch(tm, p, grid, st);
+    case 32: return GemmLauncher<FMT, 32>::launch(tm, p, grid, st);
+    case 64: return GemmLauncher<FMT, 64>::launch(tm, p, grid, st);
+    default: return GemmLauncher<FMT, 128>::launch(tm, p, grid, st);
+  }
+}
+
+#define DQ_FMT_SWITCH(fmt, CALL)                  \
+  switch (fmt) {                                  \
+    case FMT_INT4: { constexpr int F = FMT_INT4; CALL; } break;   \
+    case FMT_NVFP4: { constexpr int F = FMT_NVFP4; CALL; } break; \
+    case FMT_MXFP4: { constexpr int F = FMT_MXFP4; CALL; } break; \
+    case FMT_FP8: { constexpr int F = FMT_FP8; CALL; } break;     \
+    default: { constexpr int F = FMT_FP8S; CALL; } break;         \
+  }
+
+void fill_plan(const dqgemm_s* h, int M, dqgemm_plan* pl) {
+  std::memset(pl, 0, sizeof(*pl));
+  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  pl->bn = bn;
+  pl->m_tiles = (M + bn - 1) / bn;
+  pl->n_tiles = h->n_tiles;
+  pl->k_stages = h->k_stages;
+  const long long T = (long long)pl->m_tiles * pl->n_tiles;
+  const long long U = T * pl->k_stages;
+  const int G = (int)std::min<long long>(U, h->num_sms);
+  pl->grid = G;
+  int maxseg = 1;
+  for (long long t = 0; t < T; ++t) {
+    const int c0 = cta_of_unit(t * pl->k_stages, U, G), c1 = cta_of_unit(t * pl->k_stages + pl->k_stages - 1, U, G);
+    maxseg = std::max(maxseg, c1 - c0 + 1);
+  }
+  pl->max_segments = maxseg;
+  int st = 0, sm = 0;
+  DQ_FMT_SWITCH(h->fmt, st = stages_for<F>(bn); sm = smem_for<F>(bn));
+  pl->stages = st;
+  pl->smem_bytes = sm;
+  pl->workspace_bytes = maxseg > 1 ? (long long)G * 2 * bn * TILE_N * 4 : 0;
+  pl->weight_bytes = h->weight_bytes;
+}
+
+dqgemm_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA; }
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* dqgemm_status_string(dqgemm_status s) {
+  switch (s) {
+    case DQ_OK: return "DQ_OK";
+    case DQ_ERR_INVALID_ARG: return "DQ_ERR_INVALID_ARG";
+    case DQ_ERR_UNSUPPORTED: return "DQ_ERR_UNSUPPORTED";
+    case DQ_ERR_ALIGNMENT: return "DQ_ERR_ALIGNMENT";
+    case DQ_ERR_ALLOC: return "DQ_ERR_ALLOC";
+    case DQ_ERR_CUDA: return "DQ_ERR_CUDA";
+    case DQ_ERR_TIMEOUT: return "DQ_ERR_TIMEOUT";
+  }
+  return "DQ_ERR_UNKNOWN";
+}
+
+dqgemm_status dqgemm_destroy(dqgemm_handle h) {
+  if (!h) return DQ_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  cudaFree(h->wchunks);
+  cudaFree(h->col_scale);
+  cudaFree(h->bias);
+  cudaFree(h->status);
+  cudaFree(h->ws);
+  cudaFree(h->counters);
+  delete h;
+  return DQ_OK;
+}
+
+dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N, const void* packed_w,
+                            const void* scales, float global_scale, const void* bias) {
+  if (!out) return DQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int fmt = (int)fmt_;
+  dqgemm_status st = check_shape(fmt, K, N);
+  if (st != DQ_OK) return st;
+  if (!packed_w || !scales) return DQ_ERR_INVALID_ARG;
+  if (!aligned16(packed_w) || !aligned16(scales) || (bias && !aligned16(bias))) return DQ_ERR_ALIGNMENT;
+  if (!is_device_ptr(packed_w) || !is_device_ptr(scales) || (bias && !is_device_ptr(bias)))
+    return DQ_ERR_INVALID_ARG;
+  if ((fmt == FMT_NVFP4 || fmt == FMT_FP8S) && !(std::isfinite(global_scale) && global_scale > 0.f))
+    return DQ_ERR_INVALID_ARG;
+
+  std::vector<uint8_t> hp(packed_bytes(fmt, K, N)), hs(scale_bytes(fmt, K, N));
+  if (cudaMemcpy(hp.data(), packed_w, hp.size(), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(hs.data(), scales, hs.size(), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DQ_ERR_CUDA;
+
+  dqgemm_s* h = new dqgemm_s();
+  h->fmt = fmt;
+  h->K = K;
+  h->N = N;
+  h->k_stages = (K + STAGE_K - 1) / STAGE_K;
+  h->n_tiles = (N + TILE_N - 1) / TILE_N;
+  h->weight_bytes = (long long)(hp.size() + hs.size());
+  cudaGetDevice(&h->device);
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+
+  // epilogue factors
+  if (fmt == FMT_NVFP4) {
+    h->sigma = global_scale * 128.f;   // operand carries dec(sb) * 2^-7
+  } else if (fmt == FMT_MXFP4) {
+    int cmax = 0;
+    for (uint8_t c : hs) cmax = std::max<int>(cmax, c);
+    if (cmax == 255) { delete h; return DQ_ERR_INVALID_ARG; }   // NaN scale
+    const int J = std::max(0, cmax - 128);
+    h->mx_bias = 126 - J;
+    h->sigma = std::ldexp(1.f, J);
+  } else if (fmt == FMT_FP8S) {
+    h->sigma = global_scale;
+    h->s_x = global_scale;
+  }
+
+  std::vector<uint8_t> chunks;
+  relayout(fmt, K, N, h->k_stages, h->n_tiles, hp, hs, chunks);
+  h->wchunk_bytes = chunks.size();
+
+  cudaError_t e = cudaMalloc(&h->wchunks, chunks.size());
+  if (e == cudaSuccess) e = cudaMalloc(&h->status, sizeof(int));
+  if (e == cudaSuccess && (fmt == FMT_FP8 || fmt == FMT_FP8S)) e = cudaMalloc(&h->col_scale, (size_t)N * 4);
+  if (e == cudaSuccess && bias) e = cudaMalloc(&h->bias, (size_t)N * 2);
+  if (e != cudaSuccess) { dqgemm_destroy(h); return DQ_ERR_ALLOC; }
+  e = cudaMemcpy(h->wchunks, chunks.data(), chunks.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
+  if (e == cudaSuccess && h->col_scale) e = cudaMemcpy(h->col_scale, hs.data(), (size_t)N * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && h->bias) e = cudaMemcpy(h->bias, bias, (size_t)N * 2, cudaMemcpyDeviceToDevice);
+  if (e == cudaSuccess) { DQ_FMT_SWITCH(fmt, e = set_attrs<F>()); }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) { dqgemm_destroy(h); return DQ_ERR_CUDA; }
+  *out = h;
+  return DQ_OK;
+}
+
+dqgemm_status dqgemm_get_plan(dqgemm_handle h, int M, dqgemm_plan* plan) {
+  if (!h || !plan || M < 1) return DQ_ERR_INVALID_ARG;
+  fill_plan(h, M, plan);
+  return DQ_OK;
+}
+
+dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream) {
+  if (!h || !x || !y || M < 1) return DQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
+  dqgemm_plan pl;
+  fill_plan(h, M, &pl);
+  const size_t tiles = (size_t)pl.m_tiles * pl.n_tiles;
+  if ((size_t)pl.workspace_bytes > h->ws_bytes || (pl.max_segments > 1 && tiles > h->counters_n)) {
+    cudaDeviceSynchronize();
+    if ((size_t)pl.workspace_bytes > h->ws_bytes) {
+      cudaFree(h->ws);
+      h->ws = nullptr;
+      h->ws_bytes = 0;
+      if (cudaMalloc(&h->ws, pl.workspace_bytes) != cudaSuccess) return DQ_ERR_ALLOC;
+      h->ws_bytes = pl.workspace_bytes;
+    }
+    if (tiles > h->counters_n) {
+      cudaFree(h->counters);
+      h->counters = nullptr;
+      h->counters_n = 0;
+      if (cudaMalloc(&h->counters, tiles * sizeof(int)) != cudaSuccess) return DQ_ERR_ALLOC;
+      if (cudaMemset(h->counters, 0, tiles * sizeof(int)) != cudaSuccess) return DQ_ERR_CUDA;
+      h->counters_n = tiles;
+    }
+    if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;
+  }
+  CUtensorMap tm;
+  if (!make_x_map(&tm, x, M, h->K, pl.bn)) return DQ_ERR_CUDA;
+  GemmParams p;
+  p.wchunks = h->wchunks;
+  p.col_scale = h->col_scale;
+  p.bias = h->bias;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.ws = h->ws;
+  p.counters = h->counters;
+  p.status = h->status;
+  p.sigma = h->sigma;
+  p.s_x = h->s_x;
+  p.mx_bias = h->mx_bias;
+  p.M = M;
+  p.N = h->N;
+  p.k_stages = h->k_stages;
+  p.m_tiles = pl.m_tiles;
+  p.units = (long long)tiles * h->k_stages;
+  p.timeout_ns = timeout_ns();
+  cudaError_t e = cudaSuccess;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DQ_FMT_SWITCH(h->fmt, e = launch_fmt<F>(pl.bn, tm, p, pl.grid, s));
+  return cuda_err(e);
+}
+
+dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream) {
+  if (!h || !w_bf16) return DQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(h->n_tiles, h->k_stages);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(w_bf16);
+  // static FP8: the weight alone is e4m3 * s_w[n] (sigma there is the activation scale)
+  const float sigma = h->fmt == FMT_FP8S ? 1.f : h->sigma;
+  DQ_FMT_SWITCH(h->fmt, (dequant_kernel<F><<<grid, 256, 0, s>>>(h->wchunks, h->col_scale, sigma, h->mx_bias,
+                                                                 h->N, h->K, h->k_stages, o)));
+  return cuda_err(cudaGetLastError());
+}
+
+dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x, void* q, void* stream) {
+  if (!x || !q || M < 1 || K < 1 || !(std::isfinite(s_x) && s_x > 0.f)) return DQ_ERR_INVALID_ARG;
+  const long long count = (long long)M * K;
+  const int blocks = (int)std::min<long long>((count + 255) / 256, 148 * 8);
+  act_quant_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), count, s_x, static_cast<uint8_t*>(q));
+  return cuda_err(cudaGetLastError());
+}
+
+dqgemm_status dqgemm_pack_host(dqgemm_format fmt_, const float* W, int K, int N, void* packed, void* scales,
+                               float* global_scale) {
+  const int fmt = (int)fmt_;
+  dqgemm_status st = check_shape(fmt, K, N);
+  if (st != DQ_OK) return st;
+  if (!W || !packed || !scales) return DQ_ERR_INVALID_ARG;
+  const size_t count = (size_t)N * K;
+  float amax = 0.f;
+  for (size_t i = 0; i < count; ++i) {
+    if (!std::isfinite(W[i])) return DQ_ERR_INVALID_ARG;
+    amax = std::max(amax, std::fabs(W[i]));
+  }
+  uint8_t* P = static_cast<uint8_t*>(packed);
+  float g = 1.f;
+  std::vector<int8_t> c8(128);
+  std::vector<uint8_t> cu(128);
+  for (int n = 0; n < N; ++n) {
+    const float* w = W + (size_t)n * K;
+    if (fmt == FMT_INT4) {
+      uint16_t* S = static_cast<uint16_t*>(scales);
+      for (int gi = 0; gi < K / 128; ++gi) {
+        S[(size_t)n * (K / 128) + gi] = quant_int4_group(w + gi * 128, 128, c8.data());
+        for (int i = 0; i < 64; ++i)
+          P[(size_t)n * (K / 2) + gi * 64 + i] = (uint8_t)((c8[2 * i] & 0xF) | ((c8[2 * i + 1] & 0xF) << 4));
+      }
+    } else if (fmt == FMT_NVFP4) {
+      g = nvfp4_global_scale(amax);
+      uint8_t* S = static_cast<uint8_t*>(scales);
+      for (int b = 0; b < K / 16; ++b) {
+        S[(size_t)n * (K / 16) + b] = quant_nvfp4_block(w + b * 16, 16, g, cu.data());
+        for (int i = 0; i < 8; ++i) P[(size_t)n * (K / 2) + b * 8 + i] = (uint8_t)(cu[2 * i] | (cu[2 * i + 1] << 4));
+      }
+    } else if (fmt == FMT_MXFP4) {
+      uint8_t* S = static_cast<uint8_t*>(scales);
+      for (int b = 0; b < K / 32; ++b) {
+        S[(size_t)n * (K / 32) + b] = quant_mxfp4_block(w + b * 32, 32, cu.data());
+        for (int i = 0; i < 16; ++i)
+          P[(size_t)n * (K / 2) + b * 16 + i] = (uint8_t)(cu[2 * i] | (cu[2 * i + 1] << 4));
+      }
+    } else {
+      float* S = static_cast<float*>(scales);
+      S[n] = quant_fp8_row(w, K, P + (size_t)n * K);
+    }
+  }
+  if (global_scale) *global_scale = (fmt == FMT_NVFP4) ? nvfp4_global_scale(amax) : 1.f;
+  return DQ_OK;
+}
+
+dqgemm_status dqgemm_pack_device(dqgemm_format fmt_, const float* W, int K, int N, void* packed, void* scales,
+                                 float* global_scale, void* stream) {
+  const int fmt = (int)fmt_;
+  dqgemm_status st = check_shape(fmt, K, N);
+  if (st != DQ_OK) return st;
+  if (!W || !packed || !scales) return DQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scales)) return DQ_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* P = static_cast<uint8_t*>(packed);
+  const long long count = (long long)N * K;
+  unsigned int* amax = nullptr;
+  float* gdev = nullptr;
+  if (cudaMalloc(&amax, 8) != cudaSuccess) return DQ_ERR_ALLOC;
+  gdev = reinterpret_cast<float*>(amax + 1);
+  cudaError_t e = cudaMemsetAsync(amax, 0, 8, s);
+  const int T = 256;
+  if (fmt == FMT_INT4) {
+    const long long n = (long long)N * (K / 128);
+    pack_int4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint16_t*>(scales));
+  } else if (fmt == FMT_NVFP4) {
+    amax_kernel<<<(unsigned)std::min<long long>((count + T - 1) / T, 4096), T, 0, s>>>(W, count, amax);
+    const long long n = (long long)N * (K / 16);
+    pack_nvfp4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, amax, P, static_cast<uint8_t*>(scales),
+                                                                gdev);
+  } else if (fmt == FMT_MXFP4) {
+    const long long n = (long long)N * (K / 32);
+    pack_mxfp4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint8_t*>(scales));
+  } else {
+    pack_fp8_kernel<<<(unsigned)((N + 7) / 8), T, 0, s>>>(W, N, K, P, static_cast<float*>(scales));
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess && global_scale) {
+    float g = 1.f;
+    if (fmt == FMT_NVFP4) e = cudaMemcpyAsync(&g, gdev, 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    *global_scale = g;
+  }
+  cudaStreamSynchronize(s);
+  cudaFree(amax);
+  return cuda_err(e);
+}
+
+dqgemm_status dqgemm_last_error(dqgemm_handle h) {
+  if (!h) return DQ_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ERR_CUDA;
+  if (v != 0) {
+    cudaMemset(h->status, 0, sizeof(int));
+    // a kernel that gave up may have left split-K counters mid-count
+    if (h->counters) cudaMemset(h->counters, 0, h->counters_n * sizeof(int));
+    cudaDeviceSynchronize();
+  }
+  return v == 0 ? DQ_OK : (dqgemm_status)v;
+}
+
+dqgemm_status dqgemm_selftest_timeout(int timeout_us, void* stream) {
+  if (timeout_us < 1) return DQ_ERR_INVALID_ARG;
+  int* status = nullptr;
+  if (cudaMalloc(&status, sizeof(int)) != cudaSuccess) return DQ_ERR_ALLOC;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(status, 0xFF, sizeof(int), s);
+  selftest_timeout_kernel<<<1, 32, 0, s>>>(status, (unsigned long long)timeout_us * 1000ull);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  int v = -1;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&v, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  cudaFree(status);
+  if (e != cudaSuccess) return DQ_ERR_CUDA;
+  return v == DEV_TIMEOUT ? DQ_ERR_TIMEOUT : (v == DEV_OK ? DQ_OK : DQ_ERR_CUDA);
+}
+
+}  // extern "C"

@@ -1,0 +1,143 @@
+// dq_aux.cuh -- the non-GEMM kernels: debug dequantization through the
+// GEMM's own unpack code, the static-FP8 activation quantizer, the GPU weight
+// packer, and the bounded-wait self test.
+#pragma once
+
+#include "dq_codec.h"
+#include "dq_gemm.cuh"
+
+namespace dq {
+
+// ---------------------------------------------------------------------------
+// debug dequantization: one CTA per (tile, stage), 256 threads = 128 rows x
+// 2 k-halves, exactly the prologue's thread mapping.  The chunk is staged in
+// shared memory and unpacked by prologue_stage, then multiplied by the
+// epilogue factor of its channel: out = bf16(f32(operand) * sigma_n).
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* wchunks, const float* col_scale, float sigma,
+                                                      int mx_bias, int N, int K, int k_stages,
+                                                      __nv_bfloat16* out) {
+  __shared__ __align__(16) uint8_t chunk[chunk_bytes(FMT)];
+  const int t = blockIdx.x, s = blockIdx.y;
+  const uint8_t* src = wchunks + ((size_t)t * k_stages + s) * chunk_bytes(FMT);
+  for (int i = threadIdx.x * 16; i < chunk_bytes(FMT); i += 256 * 16)
+    *reinterpret_cast<uint4*>(chunk + i) = *reinterpret_cast<const uint4*>(src + i);
+  __syncthreads();
+  const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+  const int n = t * TILE_N + r;
+  if (n >= N) return;
+  const float sig = col_scale ? sigma * col_scale[n] : sigma;
+  if constexpr (FMT == FMT_FP8S) {
+    for (int kl = h * 64; kl < h * 64 + 64; ++kl) {
+      const int k = s * STAGE_K + kl;
+      if (k >= K) break;
+      const uint8_t c = chunk[r * 128 + (((kl >> 4) ^ (r & 7)) << 4) + (kl & 15)];
+      out[(size_t)n * K + k] = __float2bfloat16_rn(__fmul_rn(e4m3_decode(c), sig));
+    }
+  } else {
+    uint32_t o[32];
+    prologue_stage<FMT, 16>(chunk, r, h, mx_bias, o);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int k = s * STAGE_K + h * 64 + 2 * i;
+      const float lo = __uint_as_float(o[i] << 16), hi = __uint_as_float(o[i] & 0xFFFF0000u);
+      if (k < K) out[(size_t)n * K + k] = __float2bfloat16_rn(__fmul_rn(lo, sig));
+      if (k + 1 < K) out[(size_t)n * K + k + 1] = __float2bfloat16_rn(__fmul_rn(hi, sig));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// static FP8 activation quantization: q = e4m3(f32(x / s_x)), saturating
+// ---------------------------------------------------------------------------
+__global__ void act_quant_kernel(const __nv_bfloat16* x, long long count, float s_x, uint8_t* q) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float v = __fdiv_rn(__bfloat162float(x[i]), s_x);
+    uint8_t c = (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+    if ((c & 0x7F) == 0) c = signbit(v) ? 0x80 : 0x00;   // a zero keeps the sign of x
+    q[i] = c;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// GPU packer (bit-identical with the host packer: same dq_codec.h routines)
+// ---------------------------------------------------------------------------
+__global__ void pack_int4_kernel(const float* W, int N, int K, uint8_t* packed, uint16_t* scales) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int groups = K / 128;
+  if (gid >= (long long)N * groups) return;
+  const int n = (int)(gid / groups), g = (int)(gid % groups);
+  int8_t c[128];
+  scales[gid] = quant_int4_group(W + (size_t)n * K + g * 128, 128, c);
+  uint8_t* dst = packed + (size_t)n * (K / 2) + g * 64;
+  for (int i = 0; i < 64; ++i) dst[i] = (uint8_t)((c[2 * i] & 0xF) | ((c[2 * i + 1] & 0xF) << 4));
+}
+
+__global__ void amax_kernel(const float* W, long long count, unsigned int* amax_bits) {
+  float a = 0.f;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x)
+    a = fmaxf(a, fabsf(W[i]));
+  for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(a));   // a >= 0: bit order = value order
+}
+
+__global__ void pack_nvfp4_kernel(const float* W, int N, int K, const unsigned int* amax_bits, uint8_t* packed,
+                                  uint8_t* scales, float* g_out) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int blocks = K / 16;
+  const float g = nvfp4_global_scale(__uint_as_float(*amax_bits));
+  if (gid == 0 && g_out) *g_out = g;
+  if (gid >= (long long)N * blocks) return;
+  const int n = (int)(gid / blocks), b = (int)(gid % blocks);
+  uint8_t c[16];
+  scales[gid] = quant_nvfp4_block(W + (size_t)n * K + b * 16, 16, g, c);
+  uint8_t* dst = packed + (size_t)n * (K / 2) + b * 8;
+  for (int i = 0; i < 8; ++i) dst[i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+}
+
+__global__ void pack_mxfp4_kernel(const float* W, int N, int K, uint8_t* packed, uint8_t* scales) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int blocks = K / 32;
+  if (gid >= (long long)N * blocks) return;
+  const int n = (int)(gid / blocks), b = (int)(gid % blocks);
+  uint8_t c[32];
+  scales[gid] = quant_mxfp4_block(W + (size_t)n * K + b * 32, 32, c);
+  uint8_t* dst = packed + (size_t)n * (K / 2) + b * 16;
+  for (int i = 0; i < 16; ++i) dst[i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+}
+
+// one warp per row: amax by shuffle, then the codes
+__global__ void pack_fp8_kernel(const float* W, int N, int K, uint8_t* codes, float* scales) {
+  const int n = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (n >= N) return;
+  const float* w = W + (size_t)n * K;
+  float a = 0.f;
+  for (int k = lane; k < K; k += 32) a = fmaxf(a, fabsf(w[k]));
+  for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  const float s = fdiv(a, 448.f);
+  if (lane == 0) scales[n] = s;
+  for (int k = lane; k < K; k += 32) codes[(size_t)n * K + k] = s > 0.f ? e4m3_encode_sat(fdiv(w[k], s)) : 0;
+}
+
+// ---------------------------------------------------------------------------
+// bounded-wait self test: waits on a barrier nothing will ever arrive at
+// ---------------------------------------------------------------------------
+__global__ void selftest_timeout_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl ctl{&abort_flag, status, timeout_ns};
+    if (mbar_wait(&bar, 0, ctl)) atomicExch(status, DEV_OK);
+  }
+}
+
+}  // namespace dq

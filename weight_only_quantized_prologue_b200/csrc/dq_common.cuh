@@ -1,0 +1,291 @@
+// dq_common.cuh -- sm_100a building blocks shared by the kernels: mbarriers
+// with bounded waits, bulk / tensor copies, tcgen05 (TMEM, MMA, commit), the
+// shared-memory matrix descriptor, and the in-register unpack of the packed
+// weight codes into bf16x2 tensor-core operands.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dq_layout.h"
+
+namespace dq {
+
+// ---------------------------------------------------------------------------
+// device status word values (mirrors dqgemm_status)
+// ---------------------------------------------------------------------------
+constexpr int DEV_OK = 0;
+constexpr int DEV_TIMEOUT = 6;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Shared control block for bounded waits: every wait gives up after
+// `timeout_ns`, or as soon as another thread of the CTA has given up; the
+// first thread to give up records DEV_TIMEOUT in the global status word.
+struct WaitCtl {
+  volatile int* abort;   // shared memory flag
+  int* status;           // global status word (may be null)
+  uint64_t timeout_ns;
+};
+
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 31) == 0) {
+      if (*ctl.abort) return false;
+      if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+        *ctl.abort = 1;
+        if (ctl.status) atomicExch(ctl.status, DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, ctl);
+}
+
+// ---------------------------------------------------------------------------
+// bulk and tensor copies global -> shared (no multicast anywhere)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05: tensor memory and MMA
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, bf16 inputs, fp32 accumulate
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, e4m3 inputs, fp32 accumulate
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptors (M = 128 rows of W, N = BN rows of x, K-major A and B).
+__host__ __device__ constexpr uint32_t idesc_bf16(int bn) {
+  return (1u << 4)            // D format f32
+         | (1u << 7)          // A bf16
+         | (1u << 10)         // B bf16
+         | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(TILE_N >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_e4m3(int bn) {
+  return (1u << 4)  // D f32; A, B format 0 = E4M3
+         | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(TILE_N >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart.  `saddr` must lie in a
+// 1024-byte-aligned swizzle atom (plus the k offset within its row).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// TMEM stores/loads, 32 lanes x 32 bits per warp, N consecutive columns.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory vector access
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 lds128(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ void sts128(void* p, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// unpack: packed codes -> bf16x2 tensor-core operands
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                             *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                             *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// INT4: a nibble n with bits 0x4300 | (n ^ 8) is the bf16 value 136 + c for
+// the two's-complement code c; subtracting 136 is exact, and one rounding
+// multiply gives bf16(c * s) -- the page's dequantize_affine with zero-point 0.
+__device__ __forceinline__ void unpack_int4(uint32_t q, uint32_t s2, uint32_t* o) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) ^ 0x43084308u;
+    o[j] = bmul2(bsub2(v, 0x43084308u), s2);
+  }
+}
+
+// E2M1: magnitude bits (e1 e0 m) placed at bf16 bits 8..6 with the sign at
+// bit 15 read as a bf16 are exactly e2m1 * 2^-126 (the subnormal code 0.5
+// lands on a bf16 subnormal, code 0 on zero).  The block scale word s2
+// carries 2^126 times the wanted factor, so the product is exact.
+__device__ __forceinline__ void unpack_e2m1(uint32_t q, uint32_t s2, uint32_t* o) {
+  const uint32_t w0 = ((q << 6) & 0x01C001C0u) | ((q << 1) & 0x80008000u);
+  const uint32_t w1 = (q << 3) & 0x81C081C0u;
+  const uint32_t w2 = q & 0x81C081C0u;
+  const uint32_t w3 = ((q >> 3) & 0x01C001C0u) | ((q << 2) & 0x80008000u);
+  o[0] = bmul2(w0, s2);
+  o[1] = bmul2(w1, s2);
+  o[2] = bmul2(w2, s2);
+  o[3] = bmul2(w3, s2);
+}
+
+// E4M3: magnitude bits at bf16 bits 10..4 with the sign at bit 15 read as a
+// bf16 are exactly e4m3 * 2^-120; multiplying by 2^120 is exact.
+constexpr uint32_t BF16X2_2P120 = 0x7B807B80u;
+__device__ __forceinline__ void unpack_e4m3(uint32_t q, uint32_t* o) {
+  const uint32_t w0 = ((q << 4) & 0x07F007F0u) | (q & 0x80008000u);
+  const uint32_t w1 = ((q >> 3) & 0x07F007F0u) | ((q << 1) & 0x80008000u);
+  o[0] = bmul2(w0, BF16X2_2P120);
+  o[1] = bmul2(w1, BF16X2_2P120);
+}
+
+// NVFP4 block scale: bf16 of dec(sb) * 2^119 for a non-negative E4M3 code,
+// so that (e2m1 * 2^-126) * it = e2m1 * dec(sb) * 2^-7 exactly; the epilogue
+// multiplies by g * 2^7.
+__device__ __forceinline__ uint32_t nvfp4_scale_bf16(uint32_t code) {
+  const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+  const uint32_t normal = ((code & 0x7Fu) << 4) + 0x7780u;             // exponent field + 239
+  const uint32_t sub = __float_as_uint((float)m * 0x1p110f) >> 16;    // m * 2^-9 * 2^119
+  return e ? normal : sub;
+}
+
+// MXFP4 block scale: bf16 2^(e - 127) * 2^(126 - J) with the handle's shift
+// J folded into `bias` = 126 - J; fields outside the normal range clamp.
+__device__ __forceinline__ uint32_t mxfp4_scale_bf16(uint32_t code, int bias) {
+  int f = (int)code + bias;
+  f = f < 0 ? 0 : (f > 254 ? 254 : f);
+  return (uint32_t)f << 7;
+}
+
+}  // namespace dq
