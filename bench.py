@@ -223,7 +223,8 @@ def run_ours(args, rank, world, local_rank):
         # a second graph family with CUDA events around every call, for the
         # per-kernel durations behind the roofline figure
         n_ev = 2 * R
-        ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(CALLS_PER_STEP)]
+        ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+               for _ in range(CALLS_PER_STEP)]
               for _ in range(n_ev)]
         g_ev = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_ev, stream=stream):
@@ -240,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.stream(stream):
         if sampler:
             sampler.start()
-        settle_until = time.time() + 1.5          # clocks settle under load (untimed)
+        settle_until = time.time() + args.settle_seconds   # clocks settle under load (untimed)
         i = 0
         while time.time() < settle_until:
             graphs[i % R].replay()
@@ -554,6 +555,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--settle-seconds", type=float, default=1.5,
+                    help="untimed load before the warmup so clocks settle and get sampled")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--sweep-m", default="1,16,32,128,1024,4096")
     ap.add_argument("--sweep-kn", default="4096x4096,4096x14336,14336x4096")

@@ -27,11 +27,8 @@ struct dqgemm_s {
   int* status = nullptr;            // device status word
   float sigma = 1.f, s_x = 1.f;
   int mx_bias = 126;
-  float* ws = nullptr;              // split-K partials
-  size_t ws_bytes = 0;
-  int* counters = nullptr;          // per-tile arrival counters
-  size_t counters_n = 0;
   long long weight_bytes = 0;       // canonical packed + scale bytes
+  int max_clusters[4][9] = {};      // co-resident clusters per (BN index, cluster size), 0 = unknown
 };
 
 namespace {
@@ -193,15 +190,66 @@ bool make_x_map(CUtensorMap* map, const void* x, int M, int K, int bn) {
 // ---------------------------------------------------------------------------
 // launch dispatch
 // ---------------------------------------------------------------------------
+bool pdl_enabled() {
+  static bool on = [] {
+    const char* e = std::getenv("DQGEMM_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int FMT, int BN>
 struct GemmLauncher {
   using C = GemmCfg<FMT, BN>;
   static cudaError_t set_attr() {
-    return cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    // every GEMM kernel asks for the same (largest) shared-memory carveout, so
+    // back-to-back calls never reconfigure the SM's L1 / shared split
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    return e;
+  }
+  static void config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attrs, int grid, int split, cudaStream_t st) {
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    int na = 0;
+    if (pdl_enabled()) {
+      attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attrs[na].val.programmaticStreamSerializationAllowed = 1;
+      ++na;
+    }
+    if (split > 1) {
+      attrs[na].id = cudaLaunchAttributeClusterDimension;
+      attrs[na].val.clusterDim.x = split;
+      attrs[na].val.clusterDim.y = 1;
+      attrs[na].val.clusterDim.z = 1;
+      ++na;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
   }
   static cudaError_t launch(const CUtensorMap& tm, const GemmParams& p, int grid, cudaStream_t st) {
-    dq_gemm_kernel<FMT, BN><<<grid, C::THREADS, C::SMEM, st>>>(tm, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attrs[2];
+    config(cfg, attrs, grid, p.split, st);
+    return cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN>, tm, p);
+  }
+  static int max_active_clusters(int split) {
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attrs[2];
+    config(cfg, attrs, split, split, nullptr);
+    int n = 0;
+    if (split > 1) {
+      if (cudaOccupancyMaxActiveClusters(&n, dq_gemm_kernel<FMT, BN>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+    }
+    return n;
   }
 };
 
@@ -241,6 +289,16 @@ cudaError_t launch_fmt(int bn, const CUtensorMap& tm, const GemmParams& p, int g
   }
 }
 
+template <int FMT>
+int max_clusters_fmt(int bn, int split) {
+  switch (bn) {
+    case 16: return GemmLauncher<FMT, 16>::max_active_clusters(split);
+    case 32: return GemmLauncher<FMT, 32>::max_active_clusters(split);
+    case 64: return GemmLauncher<FMT, 64>::max_active_clusters(split);
+    default: return GemmLauncher<FMT, 128>::max_active_clusters(split);
+  }
+}
+
 #define DQ_FMT_SWITCH(fmt, CALL)                  \
   switch (fmt) {                                  \
     case FMT_INT4: { constexpr int F = FMT_INT4; CALL; } break;   \
@@ -250,7 +308,24 @@ cudaError_t launch_fmt(int bn, const CUtensorMap& tm, const GemmParams& p, int g
     default: { constexpr int F = FMT_FP8S; CALL; } break;         \
   }
 
-void fill_plan(const dqgemm_s* h, int M, dqgemm_plan* pl) {
+int bn_index(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
+
+// How many clusters of `split` CTAs can be resident at once (cached per handle).
+int cluster_capacity(dqgemm_s* h, int bn, int split) {
+  int& c = h->max_clusters[bn_index(bn)][split];
+  if (c == 0) {
+    int n = 0;
+    DQ_FMT_SWITCH(h->fmt, n = max_clusters_fmt<F>(bn, split));
+    c = n > 0 ? n : -1;
+  }
+  return c;
+}
+
+// Tiles of 128 output channels x bn activation rows.  With at least one tile
+// per SM, each CTA computes whole tiles (persistent loop).  With fewer tiles
+// than SMs, the K range of each tile is split over the S CTAs of a cluster,
+// S the largest split (<= 8, <= k_stages) whose T * S CTAs are all resident.
+void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
   std::memset(pl, 0, sizeof(*pl));
   const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   pl->bn = bn;
@@ -258,20 +333,21 @@ void fill_plan(const dqgemm_s* h, int M, dqgemm_plan* pl) {
   pl->n_tiles = h->n_tiles;
   pl->k_stages = h->k_stages;
   const long long T = (long long)pl->m_tiles * pl->n_tiles;
-  const long long U = T * pl->k_stages;
-  const int G = (int)std::min<long long>(U, h->num_sms);
-  pl->grid = G;
-  int maxseg = 1;
-  for (long long t = 0; t < T; ++t) {
-    const int c0 = cta_of_unit(t * pl->k_stages, U, G), c1 = cta_of_unit(t * pl->k_stages + pl->k_stages - 1, U, G);
-    maxseg = std::max(maxseg, c1 - c0 + 1);
+  int split = 1;
+  if (T < h->num_sms) {
+    for (int s = std::min(8, h->k_stages); s >= 2; --s) {
+      if (T * s > h->num_sms) continue;
+      const int cap = cluster_capacity(h, bn, s);
+      if (cap > 0 && cap >= T) { split = s; break; }
+    }
   }
-  pl->max_segments = maxseg;
+  pl->max_segments = split;
+  pl->grid = split > 1 ? (int)(T * split) : (int)std::min<long long>(T, h->num_sms);
   int st = 0, sm = 0;
   DQ_FMT_SWITCH(h->fmt, st = stages_for<F>(bn); sm = smem_for<F>(bn));
   pl->stages = st;
   pl->smem_bytes = sm;
-  pl->workspace_bytes = maxseg > 1 ? (long long)G * 2 * bn * TILE_N * 4 : 0;
+  pl->workspace_bytes = 0;
   pl->weight_bytes = h->weight_bytes;
 }
 
@@ -304,8 +380,6 @@ dqgemm_status dqgemm_destroy(dqgemm_handle h) {
   cudaFree(h->col_scale);
   cudaFree(h->bias);
   cudaFree(h->status);
-  cudaFree(h->ws);
-  cudaFree(h->counters);
   delete h;
   return DQ_OK;
 }
@@ -385,26 +459,6 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
   if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
   dqgemm_plan pl;
   fill_plan(h, M, &pl);
-  const size_t tiles = (size_t)pl.m_tiles * pl.n_tiles;
-  if ((size_t)pl.workspace_bytes > h->ws_bytes || (pl.max_segments > 1 && tiles > h->counters_n)) {
-    cudaDeviceSynchronize();
-    if ((size_t)pl.workspace_bytes > h->ws_bytes) {
-      cudaFree(h->ws);
-      h->ws = nullptr;
-      h->ws_bytes = 0;
-      if (cudaMalloc(&h->ws, pl.workspace_bytes) != cudaSuccess) return DQ_ERR_ALLOC;
-      h->ws_bytes = pl.workspace_bytes;
-    }
-    if (tiles > h->counters_n) {
-      cudaFree(h->counters);
-      h->counters = nullptr;
-      h->counters_n = 0;
-      if (cudaMalloc(&h->counters, tiles * sizeof(int)) != cudaSuccess) return DQ_ERR_ALLOC;
-      if (cudaMemset(h->counters, 0, tiles * sizeof(int)) != cudaSuccess) return DQ_ERR_CUDA;
-      h->counters_n = tiles;
-    }
-    if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;
-  }
   CUtensorMap tm;
   if (!make_x_map(&tm, x, M, h->K, pl.bn)) return DQ_ERR_CUDA;
   GemmParams p;
@@ -412,8 +466,6 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
   p.col_scale = h->col_scale;
   p.bias = h->bias;
   p.y = static_cast<__nv_bfloat16*>(y);
-  p.ws = h->ws;
-  p.counters = h->counters;
   p.status = h->status;
   p.sigma = h->sigma;
   p.s_x = h->s_x;
@@ -422,7 +474,8 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
   p.N = h->N;
   p.k_stages = h->k_stages;
   p.m_tiles = pl.m_tiles;
-  p.units = (long long)tiles * h->k_stages;
+  p.tiles = pl.m_tiles * pl.n_tiles;
+  p.split = pl.max_segments;
   p.timeout_ns = timeout_ns();
   cudaError_t e = cudaSuccess;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -548,8 +601,6 @@ dqgemm_status dqgemm_last_error(dqgemm_handle h) {
   if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ERR_CUDA;
   if (v != 0) {
     cudaMemset(h->status, 0, sizeof(int));
-    // a kernel that gave up may have left split-K counters mid-count
-    if (h->counters) cudaMemset(h->counters, 0, h->counters_n * sizeof(int));
     cudaDeviceSynchronize();
   }
   return v == 0 ? DQ_OK : (dqgemm_status)v;

@@ -9,18 +9,23 @@
 //   warp 0      producer: one 1-D bulk copy of the stage's pre-tiled weight
 //               chunk + two TMA box loads of the bf16 x tile, per stage
 //   warp 1      MMA issuer: one thread issues tcgen05.mma into a TMEM
-//               accumulator and commits stage / accumulator barriers
+//               accumulator and commits stage / operand / accumulator barriers
 //   warps 2..9  the prologue: unpack + scale the packed codes of one weight
 //               row per thread (two threads per row, one per k-half) into
 //               bf16 operands written straight to TMEM (the MMA reads A from
 //               TMEM), or, for static FP8, quantize the x tile to e4m3 into
 //               shared memory; then the epilogue (tcgen05.ld, scale, bias,
 //               bf16 cast, store).
-// Work split: stream-K over (output tile, k-stage) units, one CTA per SM;
-// a tile cut between CTAs is summed by its last-arriving CTA in a fixed
-// order (deterministic), with no spin on other CTAs.
-// Every wait is bounded (WaitCtl): on expiry the CTA drains its own copies
-// and MMAs, frees TMEM, records DEV_TIMEOUT and returns.
+// Work split: a tile of 128 output channels x BN activation rows is either
+// computed whole by one CTA (persistent loop over tiles), or its K range is
+// split over the S CTAs of a thread-block cluster whose fp32 partials are
+// summed through distributed shared memory in rank order (deterministic, no
+// global scratch).
+// Back-to-back calls overlap through programmatic dependent launch: a CTA
+// sets up and starts streaming its (read-only) weights before waiting for the
+// previous grid; it reads x and writes y only after that wait.
+// Every mbarrier wait is bounded (WaitCtl): on expiry the CTA drains its own
+// copies and MMAs, frees TMEM, records DEV_TIMEOUT and returns.
 #pragma once
 
 #include "dq_common.cuh"
@@ -32,14 +37,13 @@ struct GemmParams {
   const float* col_scale;        // per output channel factor (FP8 formats) or null
   const __nv_bfloat16* bias;     // [N] or null
   __nv_bfloat16* y;              // [M, N]
-  float* ws;                     // split-K partials: [grid][2][BN][128] fp32
-  int* counters;                 // [tiles] arrival counters, self-resetting
   int* status;                   // device status word
   float sigma;                   // epilogue factor common to all channels
   float s_x;                     // static FP8 activation scale
   int mx_bias;                   // MXFP4: 126 - J
   int M, N, k_stages, m_tiles;
-  long long units;               // tiles * k_stages
+  int tiles;                     // n_tiles * m_tiles
+  int split;                     // CTAs per tile (cluster size); 1 = whole tiles
   unsigned long long timeout_ns;
 };
 
@@ -58,26 +62,56 @@ struct GemmCfg {
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);
   static constexpr int W_OFF = Q_OFF + align_up(Q_BYTES, 1024);
   static constexpr int STAGE_BYTES = W_OFF + align_up(CHUNK, 1024);
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  // skinny tiles keep a CTA under half an SM's shared memory so that the next
+  // call's CTA can be resident alongside (programmatic dependent launch)
+  static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : 200 * 1024;
+  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 6 ? 6 : STAGES_RAW);
-  static constexpr int A_COLS = STATIC ? 0 : STAGES * (STAGE_K / 2);   // bf16 A ring in TMEM
+  // TMEM: a ring of bf16 A operands plus NACC independent fp32 accumulators;
+  // the k-steps of a stage rotate over the accumulators so consecutive MMAs
+  // do not wait on each other, and the epilogue sums them in a fixed order.
+  static constexpr int TMEM_BUDGET = BN <= 64 ? 256 : 512;   // <= 256: two CTAs per SM
+  static constexpr int A_STAGES = STATIC ? 0 : (BN == 32 ? 2 : (BN == 64 ? 2 : 3));
+  static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
+  static constexpr int NACC = BN == 16 ? 4 : (BN == 32 ? 4 : 2);
   static constexpr int ACC_COL = A_COLS;
-  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + BN);
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + NACC * BN);
+  static constexpr int RED_BYTES = BN * TILE_N * 4;        // split-K partial, reuses the stage buffers
+  static constexpr int BAR_BYTES = 8 * (2 * 6 + 2 * 6 + 3) + 16;
   static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;   // + alignment slack
   static constexpr uint32_t IDESC = STATIC ? idesc_e4m3(BN) : idesc_bf16(BN);
   static constexpr uint32_t TX_BYTES = CHUNK + X_BYTES;
   static constexpr int THREADS = 320;
-  static_assert(A_COLS + BN <= 512, "TMEM budget");
+  static_assert(A_COLS + NACC * BN <= TMEM_BUDGET, "TMEM budget");
+  static_assert(RED_BYTES <= STAGES * STAGE_BYTES, "split-K partial must fit the stage buffers");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
-// CTA that owns stream-K unit u when U units are cut into G contiguous ranges
-// [floor(c U / G), floor((c+1) U / G)).
-__host__ __device__ inline int cta_of_unit(long long u, long long U, int G) {
-  return (int)(((u + 1) * (long long)G - 1) / U);
+// The work of one CTA: a list of (tile, k_begin, k_end) segments.
+struct Work {
+  int first_tile, tile_step, ntiles;  // tiles first_tile + i * tile_step, i < ntiles
+  int kb, ke;                         // k-stage range within every tile
+  __device__ int stages() const { return ntiles * (ke - kb); }
+};
+
+__device__ __forceinline__ Work cta_work(const GemmParams& p) {
+  Work w;
+  if (p.split > 1) {
+    const int q = (int)cluster_rank();
+    w.first_tile = blockIdx.x / p.split;
+    w.tile_step = 1;
+    w.ntiles = 1;
+    w.kb = (int)((unsigned)(q * p.k_stages) / (unsigned)p.split);
+    w.ke = (int)((unsigned)((q + 1) * p.k_stages) / (unsigned)p.split);
+  } else {
+    w.first_tile = blockIdx.x;
+    w.tile_step = gridDim.x;
+    w.ntiles = (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    w.kb = 0;
+    w.ke = p.k_stages;
+  }
+  return w;
 }
-__host__ __device__ inline long long cta_start(int c, long long U, int G) { return (long long)c * U / G; }
 
 template <int FMT, int BN>
 __device__ __forceinline__ void prologue_stage(const uint8_t* chunk, int r, int h, int mx_bias, uint32_t (&o)[32]) {
@@ -165,22 +199,20 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
 }
 
 template <int FMT, int BN>
-__global__ void __launch_bounds__(320, 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
+__global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                           const GemmParams p) {
   using C = GemmCfg<FMT, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* aready = full + C::STAGES;
-  uint64_t* empty = aready + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);   // smem stage loaded
+  uint64_t* empty = full + C::STAGES;                                                // smem stage consumed
+  uint64_t* aready = empty + C::STAGES;   // operand ready: TMEM A slot (bf16) / shared e4m3 x (static)
+  uint64_t* aempty = aready + 6;          // TMEM A slot consumed
+  uint64_t* acc_full = aempty + 6;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* epi_a = acc_empty + 1;
-  uint64_t* epi_b = epi_a + 1;
-  uint64_t* drain = epi_b + 1;
+  uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* bcast = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
@@ -188,16 +220,16 @@ __global__ void __launch_bounds__(320, 1) dq_gemm_kernel(const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&aready[s], 8);
       mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 6; ++a) {
+      mbar_init(&aready[a], 8);
+      mbar_init(&aempty[a], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
-    mbar_init(epi_a, 256);
-    mbar_init(epi_b, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
-    *bcast = 0;
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -206,79 +238,90 @@ __global__ void __launch_bounds__(320, 1) dq_gemm_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();   // the next call may start its own prologue now
 
-  const long long U = p.units;
-  const int G = gridDim.x;
+  const Work wk = cta_work(p);
   const int KS = p.k_stages;
-  const long long u0 = cta_start(blockIdx.x, U, G), u1 = cta_start(blockIdx.x + 1, U, G);
+  const int nst = wk.ke - wk.kb;   // stages per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      for (long long u = u0; ok && u < u1;) {
-        const int tile = (int)(u / KS), kb = (int)(u % KS);
-        const int ke = (int)((long long)kb + (u1 - u) < KS ? kb + (u1 - u) : KS);
-        const int n_tile = tile / p.m_tiles, m_tile = tile % p.m_tiles;
-        for (int ks = kb; ks < ke; ++ks, ++it) {
-          const int slot = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
-          uint8_t* st = smem + slot * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[slot], C::TX_BYTES);
-          bulk_g2s(st + C::W_OFF, p.wchunks + ((size_t)n_tile * KS + ks) * C::CHUNK, C::CHUNK, &full[slot]);
-          tma_load_2d(st + C::X_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full[slot]);
-          tma_load_2d(st + C::X_OFF + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full[slot]);
-        }
-        u += ke - kb;
+      const int total = wk.stages();
+      const int pre = total < C::STAGES ? total : C::STAGES;
+      // weights do not depend on earlier grids: stream the first stages now
+      for (int it = 0; it < pre; ++it) {
+        const int tile = wk.first_tile + (it / nst) * wk.tile_step, ks = wk.kb + it % nst;
+        mbar_arrive_expect_tx(&full[it], C::TX_BYTES);
+        bulk_g2s(smem + it * C::STAGE_BYTES + C::W_OFF,
+                 p.wchunks + ((size_t)(tile / p.m_tiles) * KS + ks) * C::CHUNK, C::CHUNK, &full[it]);
       }
-      // Never leave with copies in flight: wait for the last issued stages
-      // (their full barriers complete on data arrival alone).
+      pdl_wait();   // x may be the previous grid's output
+      bool ok = true;
+      int it = 0;
+      for (; ok && it < total; ++it) {
+        const int tile = wk.first_tile + (it / nst) * wk.tile_step, ks = wk.kb + it % nst;
+        const int m_tile = tile % p.m_tiles;
+        const int slot = it % C::STAGES;
+        uint8_t* st = smem + slot * C::STAGE_BYTES;
+        if (it >= pre) {
+          if (!mbar_wait(&empty[slot], ((it / C::STAGES) & 1) ^ 1, ctl)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[slot], C::TX_BYTES);
+          bulk_g2s(st + C::W_OFF, p.wchunks + ((size_t)(tile / p.m_tiles) * KS + ks) * C::CHUNK, C::CHUNK,
+                   &full[slot]);
+        }
+        tma_load_2d(st + C::X_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full[slot]);
+        tma_load_2d(st + C::X_OFF + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full[slot]);
+      }
+      // Never leave with copies in flight: wait for the stages issued last
+      // (a full barrier completes on data arrival alone; the loop only stops
+      // early after `pre`, so every prefetched stage got its x tile too).
       volatile int no_abort = 0;
       const WaitCtl drain_ctl{&no_abort, p.status, p.timeout_ns};
-      const uint32_t first = it > (uint32_t)C::STAGES ? it - C::STAGES : 0;
-      for (uint32_t i = first; i < it; ++i) mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
+      const int issued = it > pre ? it : pre;
+      const int first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (int i = first; i < issued; ++i) mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t it = 0;
-      int seg = 0;
+      int it = 0;
       bool ok = true;
-      for (long long u = u0; ok && u < u1; ++seg) {
-        const int kb = (int)(u % KS);
-        const int ke = (int)((long long)kb + (u1 - u) < KS ? kb + (u1 - u) : KS);
-        if (!mbar_wait(acc_empty, (seg & 1) ^ 1, ctl)) break;
+      for (int t = 0; ok && t < wk.ntiles; ++t) {
+        if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl)) break;
         tc_fence_after();
-        for (int ks = kb; ks < ke; ++ks, ++it) {
+        for (int j = 0; j < nst; ++j, ++it) {
           const int slot = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait(&full[slot], ph, ctl) || !mbar_wait(&aready[slot], ph, ctl)) { ok = false; break; }
-          tc_fence_after();
+          if (!mbar_wait(&full[slot], ph, ctl)) { ok = false; break; }
           uint8_t* st = smem + slot * C::STAGE_BYTES;
           if constexpr (!C::STATIC) {
+            const int as = it % C::A_STAGES;
+            if (!mbar_wait(&aready[as], (it / C::A_STAGES) & 1, ctl)) { ok = false; break; }
+            tc_fence_after();
             const uint32_t xb = smem_u32(st + C::X_OFF);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t bd = sdesc_sw128(xb + (kk >> 2) * BN * 128 + (kk & 3) * 32);
-              mma_bf16_ts(tmem + C::ACC_COL, tmem + slot * (STAGE_K / 2) + kk * 8, bd, C::IDESC,
-                          (ks > kb || kk > 0) ? 1u : 0u);
+              mma_bf16_ts(tmem + C::ACC_COL + (kk % C::NACC) * BN, tmem + as * (STAGE_K / 2) + kk * 8, bd,
+                          C::IDESC, (j > 0 || kk >= C::NACC) ? 1u : 0u);
             }
+            tc_commit(&aempty[as]);
           } else {
+            if (!mbar_wait(&aready[slot], ph, ctl)) { ok = false; break; }
+            tc_fence_after();
             const uint32_t wb = smem_u32(st + C::W_OFF), qb = smem_u32(st + C::Q_OFF);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              mma_f8_ss(tmem + C::ACC_COL, sdesc_sw128(wb + kk * 32), sdesc_sw128(qb + kk * 32), C::IDESC,
-                        (ks > kb || kk > 0) ? 1u : 0u);
+              mma_f8_ss(tmem + C::ACC_COL + (kk % C::NACC) * BN, sdesc_sw128(wb + kk * 32),
+                        sdesc_sw128(qb + kk * 32), C::IDESC, (j > 0 || kk >= C::NACC) ? 1u : 0u);
             }
           }
           tc_commit(&empty[slot]);
         }
         if (!ok) break;
         tc_commit(acc_full);
-        u += ke - kb;
       }
       // all MMAs this thread issued must finish before TMEM is released
       volatile int no_abort = 0;
@@ -294,95 +337,64 @@ __global__ void __launch_bounds__(320, 1) dq_gemm_kernel(const __grid_constant__
     const int h = dw >> 2;              // k-half of the stage / column half of the tile
     const int r = qd * 32 + lane;       // weight row in the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
-    uint32_t it = 0;
-    int seg = 0, pseg = 0;
+    int it = 0;
     bool ok = true;
-    for (long long u = u0; ok && u < u1; ++seg) {
-      const int tile = (int)(u / KS), kb = (int)(u % KS);
-      const int ke = (int)((long long)kb + (u1 - u) < KS ? kb + (u1 - u) : KS);
-      const int n_tile = tile / p.m_tiles, m_tile = tile % p.m_tiles;
-      for (int ks = kb; ks < ke; ++ks, ++it) {
-        const int slot = it % C::STAGES;
-        const uint32_t ph = (it / C::STAGES) & 1;
-        if (!mbar_wait(&full[slot], ph, ctl)) { ok = false; break; }
-        uint8_t* st = smem + slot * C::STAGE_BYTES;
-        if constexpr (!C::STATIC) {
-          // the TMEM A slot is free once the MMAs of its previous use completed
-          if (!mbar_wait(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
-          tc_fence_after();
+    for (int t = 0; ok && t < wk.ntiles; ++t) {
+      const int tile = wk.first_tile + t * wk.tile_step;
+      if constexpr (!C::STATIC) {
+        for (int j = 0; j < nst; ++j, ++it) {
+          const int slot = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait_warp(&full[slot], ph, ctl)) { ok = false; break; }
           uint32_t o[32];
-          prologue_stage<FMT, BN>(st + C::W_OFF, r, h, p.mx_bias, o);
-          tmem_st32(tmem + lane_base + slot * (STAGE_K / 2) + h * 32, o);
+          prologue_stage<FMT, BN>(smem + slot * C::STAGE_BYTES + C::W_OFF, r, h, p.mx_bias, o);
+          const int as = it % C::A_STAGES;
+          if (!mbar_wait_warp(&aempty[as], ((it / C::A_STAGES) & 1) ^ 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          tmem_st32(tmem + lane_base + as * (STAGE_K / 2) + h * 32, o);
           tmem_wait_st();
           tc_fence_before();
-        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&aready[as]);
+        }
+      } else {
+        for (int j = 0; j < nst; ++j, ++it) {
+          const int slot = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1;
+          if (!mbar_wait_warp(&full[slot], ph, ctl)) { ok = false; break; }
+          // the shared B buffer of this slot is free once its previous MMAs finished
+          if (!mbar_wait_warp(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
+          uint8_t* st = smem + slot * C::STAGE_BYTES;
           quantize_x_tile<BN>(st + C::X_OFF, st + C::Q_OFF, p.s_x, threadIdx.x - 64);
           fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&aready[slot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&aready[slot]);
       }
       if (!ok) break;
 
-      // ---- epilogue of this segment
-      if (!mbar_wait(acc_full, seg & 1, ctl)) break;
+      // ---- epilogue of this tile
+      if (!mbar_wait_warp(acc_full, t & 1, ctl)) { ok = false; break; }
       tc_fence_after();
       constexpr int HALF = BN / 2;
       float acc[HALF];
 #pragma unroll
-      for (int c8 = 0; c8 < HALF / 8; ++c8) {
-        float v[8];
-        tmem_ld8(tmem + lane_base + C::ACC_COL + h * HALF + c8 * 8, v);
+      for (int a = 0; a < C::NACC; ++a) {
+        float v[HALF];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[c8 * 8 + i] = v[i];
+        for (int c8 = 0; c8 < HALF / 8; ++c8)
+          tmem_ld8(tmem + lane_base + C::ACC_COL + a * BN + h * HALF + c8 * 8,
+                   *reinterpret_cast<float(*)[8]>(v + c8 * 8));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) acc[i] = a == 0 ? v[i] : acc[i] + v[i];
       }
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
-
-      const long long tu = (long long)tile * KS;
-      const int c_first = cta_of_unit(tu, U, G), c_last = cta_of_unit(tu + KS - 1, U, G);
-      const int nseg = c_last - c_first + 1;
-      bool store = true;
-      if (nseg > 1) {
-        // write this CTA's partial, then let the last arriver of the tile sum
-        const int which = (seg == 0) ? 0 : 1;
-        float* mine = p.ws + ((size_t)(blockIdx.x * 2 + which) * BN) * TILE_N;
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) mine[(h * HALF + i) * TILE_N + r] = acc[i];
-        __threadfence();
-        mbar_arrive(epi_a);
-        if (dw == 0 && lane == 0) {
-          int last = 0;
-          if (mbar_wait(epi_a, pseg & 1, ctl)) {
-            const int old = atomicAdd(&p.counters[tile], 1);
-            last = (old == nseg - 1);
-            if (last) p.counters[tile] = 0;   // every contributor has arrived: reset for the next call
-          }
-          *bcast = last;
-          mbar_arrive(epi_b);
-        }
-        if (!mbar_wait(epi_b, pseg & 1, ctl)) break;
-        ++pseg;
-        store = (*bcast != 0);
-        if (store) {
-          // sum every contributor's partial (this CTA's included, re-read from
-          // the workspace) in CTA order: the result does not depend on which
-          // CTA arrived last
-          __threadfence();
-          for (int c = c_first; c <= c_last; ++c) {
-            const int w = ((cta_start(c, U, G) / KS) == tile) ? 0 : 1;
-            const float* src = p.ws + ((size_t)(c * 2 + w) * BN) * TILE_N + r;
-#pragma unroll
-            for (int i = 0; i < HALF; ++i) {
-              const float v = __ldcg(src + (h * HALF + i) * TILE_N);
-              acc[i] = (c == c_first) ? v : acc[i] + v;
-            }
-          }
-        }
-      }
-      if (store) {
+      pdl_wait();   // y (and everything after) may be read by an earlier grid
+      if (p.split == 1) {
+        const int n_tile = tile / p.m_tiles, m_tile = tile % p.m_tiles;
         const int n = n_tile * TILE_N + r;
         if (n < p.N) {
           const float sig = p.col_scale ? p.sigma * p.col_scale[n] : p.sigma;
@@ -393,9 +405,54 @@ __global__ void __launch_bounds__(320, 1) dq_gemm_kernel(const __grid_constant__
             if (m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(acc[i], sig, b));
           }
         }
+      } else {
+        // split-K partial into this CTA's shared memory: [column][row]
+        float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) red[(h * HALF + i) * TILE_N + r] = acc[i];
       }
-      u += ke - kb;
     }
+    if (!ok) *abort_flag = 1;
+  }
+
+  if (p.split > 1) {
+    // ---- cluster split-K: every CTA of the cluster reaches both barriers
+    // (all 320 threads, whether or not their work completed)
+    __syncwarp();
+    cluster_sync();
+    if (warp >= 2 && !*abort_flag) {
+      const int S = p.split;
+      const int q = (int)cluster_rank();
+      const int tile = blockIdx.x / S;
+      const int n_tile = tile / p.m_tiles, m_tile = tile % p.m_tiles;
+      // rank q finishes a slice of the tile's (column, row-quad) cells
+      const int cells = BN * (TILE_N / 4);
+      const int c0 = q * cells / S, c1 = (q + 1) * cells / S;
+      const float* red = reinterpret_cast<const float*>(smem);
+      for (int c = c0 + (int)threadIdx.x - 64; c < c1; c += 256) {
+        const int col = c / (TILE_N / 4), r4 = (c % (TILE_N / 4)) * 4;
+        float4 sum = ld_dsmem_f32x4(red + col * TILE_N + r4, 0);
+        for (int pr = 1; pr < S; ++pr) {
+          const float4 v = ld_dsmem_f32x4(red + col * TILE_N + r4, pr);
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
+        const int m = m_tile * BN + col;
+        if (m < p.M) {
+          const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int n = n_tile * TILE_N + r4 + e;
+            if (n < p.N) {
+              const float sig = p.col_scale ? p.sigma * p.col_scale[n] : p.sigma;
+              const float b = p.bias ? __bfloat162float(p.bias[n]) : 0.f;
+              p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(vals[e], sig, b));
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync();   // no CTA leaves while a peer may still read its partial
   }
 
   tc_fence_before();
