@@ -89,12 +89,15 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt, int K, int N,
                             float global_scale, const void* bias);
 
 /* y = x . deq(W)^T + b.  x: device bf16 [M, K]; y: device bf16 [M, N]; M >= 1.
- * One kernel launch on `stream`.  For DQ_FP8_STATIC the activation is
- * quantized to e4m3 inside the same kernel.  The handle owns a split-K
- * workspace that grows on the first call with a larger M (that call
- * allocates and synchronizes); calls on one handle must not overlap on
- * different streams.  Device-side wait timeouts are reported through
- * dqgemm_last_error after the stream has been synchronized. */
+ * One kernel launch on `stream` (no allocation, no synchronization).  For
+ * DQ_FP8_STATIC the activation is quantized to e4m3 inside the same kernel.
+ * When there are fewer output tiles than SMs the K range of a tile is split
+ * over a thread-block cluster whose partial sums meet in distributed shared
+ * memory (deterministic).  Launched with programmatic dependent launch: the
+ * kernel streams its weights before waiting for the previous kernel in the
+ * stream, and reads x / writes y only after that wait.  Device-side wait
+ * timeouts are reported through dqgemm_last_error after the stream has been
+ * synchronized. */
 dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream);
 
 /* Release the handle and its device memory (synchronizes the device). */
@@ -130,10 +133,28 @@ dqgemm_status dqgemm_pack_host(dqgemm_format fmt, const float* W, int K, int N,
 /* Same as dqgemm_pack_host on the GPU: W, packed and scales are device
  * pointers; results are bit-identical to dqgemm_pack_host.  If
  * `global_scale` (host pointer) is not NULL the call synchronizes `stream`
- * and stores g there.  Allocates and frees 4 bytes of device memory. */
+ * and stores g there.  Allocates and frees 8 bytes of device memory. */
 dqgemm_status dqgemm_pack_device(dqgemm_format fmt, const float* W, int K, int N,
                                  void* packed, void* scales, float* global_scale,
                                  void* stream);
+
+/* dqgemm_pack_device without any device allocation, for callers that cannot
+ * call cudaMalloc: a serving process that reserved all device memory up
+ * front, or code that must not trigger the device-wide synchronization that
+ * cudaMalloc / cudaFree may cause while other streams run.  The tutorial
+ * pages have no counterpart; this is a deployment variant of the packer.
+ * Results are bit-identical to dqgemm_pack_device.  NVFP4 needs a tensor-wide
+ * amax: its two-pass reduction keeps up to 4096 partial maxima (one per
+ * 65536 weights) in a static device array that every GPU loading the library
+ * holds (16 KB) until exit, so NVFP4 requires N*K <= 4096*65536 and returns
+ * DQ_ERR_UNSUPPORTED beyond that; the other formats need no scratch.  The
+ * first call on a device looks up the array's device address (do it before
+ * any stream capture).  All calls share the array: calls whose kernels
+ * overlap on the GPU race with each other.  If `global_scale` (host) is not
+ * NULL the call synchronizes `stream` and stores g there. */
+dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt, const float* W, int K, int N,
+                                         void* packed, void* scales, float* global_scale,
+                                         void* stream);
 
 /* Status of the last device-side check of the handle's kernels (DQ_OK or
  * DQ_ERR_TIMEOUT), then clears it.  Synchronizes the device. */

@@ -20,6 +20,7 @@ from ._native import (  # noqa: F401
     dqgemm_get_plan,
     dqgemm_last_error,
     dqgemm_pack_device,
+    dqgemm_pack_device_noalloc,
     dqgemm_pack_host,
     dqgemm_quantize_act_fp8,
     dqgemm_run,

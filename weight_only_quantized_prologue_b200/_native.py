@@ -46,6 +46,7 @@ _SIGNATURES = {
     "dqgemm_quantize_act_fp8": [_VP, _I, _I, _F, _VP, _VP],
     "dqgemm_pack_host": [_I, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_F)],
     "dqgemm_pack_device": [_I, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_F), _VP],
+    "dqgemm_pack_device_noalloc": [_I, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_F), _VP],
     "dqgemm_last_error": [_VP],
     "dqgemm_selftest_timeout": [_I, _VP],
     "dqgemm_get_plan": [_VP, _I, ctypes.POINTER(Plan)],
@@ -151,6 +152,15 @@ def dqgemm_pack_device(fmt, W, packed, scales, stream=None):
     g = ctypes.c_float(0.0)
     _check(lib().dqgemm_pack_device(FORMATS[fmt], _ptr(W), K, N, _ptr(packed), _ptr(scales), ctypes.byref(g),
                                     _stream(stream)), "dqgemm_pack_device")
+    return float(g.value)
+
+
+def dqgemm_pack_device_noalloc(fmt, W, packed, scales, stream=None):
+    """As dqgemm_pack_device, with no device allocation (static scratch)."""
+    N, K = W.shape
+    g = ctypes.c_float(0.0)
+    _check(lib().dqgemm_pack_device_noalloc(FORMATS[fmt], _ptr(W), K, N, _ptr(packed), _ptr(scales),
+                                            ctypes.byref(g), _stream(stream)), "dqgemm_pack_device_noalloc")
     return float(g.value)
 
 

@@ -594,6 +594,87 @@ dqgemm_status dqgemm_pack_device(dqgemm_format fmt_, const float* W, int K, int 
   return cuda_err(e);
 }
 
+// ---------------------------------------------------------------------------
+// allocation-free GPU packer: the NVFP4 tensor-amax scratch lives in a
+// file-scope device array instead of cudaMalloc'd memory
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kNoAllocMaxPartials = 4096;          // partial maxima the scratch holds
+constexpr long long kNoAllocChunk = 65536;         // weights reduced per partial
+// [0, 4096): partial maxima; [4096]: amax bits; [4097]: global scale g
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxPartials + 2];
+
+constexpr int kMaxDevices = 64;
+float* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch on the current device, looked up once per
+// device (the symbol's host-side name is not a device address).
+float* noalloc_scratch(dqgemm_status* st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = DQ_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      *st = DQ_ERR_CUDA;
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *st = DQ_OK;
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt_, const float* W, int K, int N, void* packed,
+                                         void* scales, float* global_scale, void* stream) {
+  const int fmt = (int)fmt_;
+  dqgemm_status st = check_shape(fmt, K, N);
+  if (st != DQ_OK) return st;
+  if (!W || !packed || !scales) return DQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(scales)) return DQ_ERR_ALIGNMENT;
+  const long long count = (long long)N * K;
+  const long long nparts = (count + kNoAllocChunk - 1) / kNoAllocChunk;
+  if (fmt == FMT_NVFP4 && nparts > kNoAllocMaxPartials) return DQ_ERR_UNSUPPORTED;   // N*K > 2^28
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* P = static_cast<uint8_t*>(packed);
+  const int T = 256;
+  cudaError_t e = cudaSuccess;
+  float g = 1.f;
+  if (fmt == FMT_INT4) {
+    const long long n = (long long)N * (K / 128);
+    pack_int4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint16_t*>(scales));
+  } else if (fmt == FMT_NVFP4) {
+    float* scratch = noalloc_scratch(&st);
+    if (!scratch) return st;
+    unsigned int* amax = reinterpret_cast<unsigned int*>(scratch + kNoAllocMaxPartials);
+    float* gdev = scratch + kNoAllocMaxPartials + 1;
+    // every scratch word read below is written earlier in the same call
+    amax_partials_kernel<<<(unsigned)nparts, T, 0, s>>>(W, count, kNoAllocChunk, scratch);
+    amax_final_kernel<<<1, T, 0, s>>>(scratch, (int)nparts, amax);
+    const long long n = (long long)N * (K / 16);
+    pack_nvfp4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, amax, P, static_cast<uint8_t*>(scales),
+                                                                gdev);
+    e = cudaGetLastError();
+    if (e == cudaSuccess && global_scale) e = cudaMemcpyAsync(&g, gdev, 4, cudaMemcpyDeviceToHost, s);
+  } else if (fmt == FMT_MXFP4) {
+    const long long n = (long long)N * (K / 32);
+    pack_mxfp4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint8_t*>(scales));
+  } else {
+    pack_fp8_kernel<<<(unsigned)((N + 7) / 8), T, 0, s>>>(W, N, K, P, static_cast<float*>(scales));
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess && global_scale) {
+    e = cudaStreamSynchronize(s);
+    *global_scale = g;
+  }
+  return cuda_err(e);
+}
+
 dqgemm_status dqgemm_last_error(dqgemm_handle h) {
   if (!h) return DQ_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;

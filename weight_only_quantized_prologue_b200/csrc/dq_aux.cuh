@@ -122,6 +122,36 @@ __global__ void pack_fp8_kernel(const float* W, int N, int K, uint8_t* codes, fl
   for (int k = lane; k < K; k += 32) codes[(size_t)n * K + k] = s > 0.f ? e4m3_encode_sat(fdiv(w[k], s)) : 0;
 }
 
+// two-pass tensor amax over fixed-size chunks (used by the allocation-free
+// packer): pass 1 writes one partial maximum per chunk, pass 2 reduces them
+__global__ void amax_partials_kernel(const float* W, long long count, long long chunk, float* partials) {
+  const long long b0 = blockIdx.x * chunk;
+  const long long b1 = b0 + chunk < count ? b0 + chunk : count;
+  float a = 0.f;
+  for (long long i = b0 + threadIdx.x; i < b1; i += blockDim.x) a = fmaxf(a, fabsf(W[i]));
+  for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  __shared__ float wmax[32];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) a = fmaxf(a, wmax[w]);
+    partials[blockIdx.x] = a;
+  }
+}
+
+__global__ void amax_final_kernel(const float* partials, int n, unsigned int* amax_bits) {
+  float a = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) a = fmaxf(a, partials[i]);
+  for (int o = 16; o; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  __shared__ float wmax[32];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) a = fmaxf(a, wmax[w]);
+    *amax_bits = __float_as_uint(a);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // bounded-wait self test: waits on a barrier nothing will ever arrive at
 // ---------------------------------------------------------------------------
