@@ -175,9 +175,21 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_x_map(CUtensorMap* map, const void* x, int M, int K, int bn) {
+// With K a multiple of 64 the map is 3-D {64, M, K/64} (the k-blocks are
+// 128 bytes apart) so one box {64, bn, 2} brings a whole 128-k stage.
+bool make_x_map(CUtensorMap* map, const void* x, int M, int K, int bn, bool* is3d) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  *is3d = (K % 64) == 0;
+  if (*is3d) {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)bn, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
   const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)bn};
@@ -333,10 +345,24 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
   pl->n_tiles = h->n_tiles;
   pl->k_stages = h->k_stages;
   const long long T = (long long)pl->m_tiles * pl->n_tiles;
+  // CTAs per SM the split may assume (skinny tiles fit two per SM)
+  static const int occ = [] {
+    const char* e = std::getenv("DQGEMM_CTAS_PER_SM");
+    const int v = e ? std::atoi(e) : 1;
+    return v >= 2 ? 2 : 1;
+  }();
+  const int slots = h->num_sms * (bn <= 64 ? occ : 1);
+  static const int force_split = [] {
+    const char* e = std::getenv("DQGEMM_SPLIT");
+    return e ? std::atoi(e) : 0;
+  }();
   int split = 1;
-  if (T < h->num_sms) {
+  if (force_split >= 1 && force_split <= 8) {
+    split = std::min(force_split, h->k_stages);
+    if (split > 1 && cluster_capacity(h, bn, split) < T) split = 1;
+  } else if (T < slots) {
     for (int s = std::min(8, h->k_stages); s >= 2; --s) {
-      if (T * s > h->num_sms) continue;
+      if (T * s > slots) continue;
       const int cap = cluster_capacity(h, bn, s);
       if (cap > 0 && cap >= T) { split = s; break; }
     }
@@ -460,7 +486,8 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
   dqgemm_plan pl;
   fill_plan(h, M, &pl);
   CUtensorMap tm;
-  if (!make_x_map(&tm, x, M, h->K, pl.bn)) return DQ_ERR_CUDA;
+  bool x3d = false;
+  if (!make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
   GemmParams p;
   p.wchunks = h->wchunks;
   p.col_scale = h->col_scale;
@@ -476,6 +503,7 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
   p.m_tiles = pl.m_tiles;
   p.tiles = pl.m_tiles * pl.n_tiles;
   p.split = pl.max_segments;
+  p.x3d = x3d ? 1 : 0;
   p.timeout_ns = timeout_ns();
   cudaError_t e = cudaSuccess;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

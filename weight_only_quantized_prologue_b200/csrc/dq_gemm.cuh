@@ -44,6 +44,7 @@ struct GemmParams {
   int M, N, k_stages, m_tiles;
   int tiles;                     // n_tiles * m_tiles
   int split;                     // CTAs per tile (cluster size); 1 = whole tiles
+  int x3d;                       // x map is 3-D {64, M, K/64}: one box per stage
   unsigned long long timeout_ns;
 };
 
@@ -56,34 +57,39 @@ template <int FMT, int BN>
 struct GemmCfg {
   static constexpr bool STATIC = (FMT == FMT_FP8S);
   static constexpr int CHUNK = chunk_bytes(FMT);
-  static constexpr int X_BYTES = BN * 256;                 // two 64-k boxes of BN rows x 128 B
+  static constexpr int X_BYTES = BN * 256;                 // two 64-k blocks of BN rows x 128 B
   static constexpr int Q_BYTES = STATIC ? BN * 128 : 0;    // e4m3 x tile (static FP8)
   static constexpr int X_OFF = 0;
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);
   static constexpr int W_OFF = Q_OFF + align_up(Q_BYTES, 1024);
   static constexpr int STAGE_BYTES = W_OFF + align_up(CHUNK, 1024);
+  // split-K receive buffer: partials pushed by the cluster's CTAs,
+  // [rank][column of this CTA's share (at most BN/2 + 1... bounded by BN/S+1)][row]
+  static constexpr int RECV_COLS = BN + 8;                 // >= S * ceil(BN / S) for S <= 8
+  static constexpr int RECV_BYTES = RECV_COLS * TILE_N * 4;
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
   static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : 200 * 1024;
-  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
+  static constexpr int STAGES_RAW = (SMEM_BUDGET - RECV_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 6 ? 6 : STAGES_RAW);
-  // TMEM: a ring of bf16 A operands plus NACC independent fp32 accumulators;
-  // the k-steps of a stage rotate over the accumulators so consecutive MMAs
-  // do not wait on each other, and the epilogue sums them in a fixed order.
-  static constexpr int TMEM_BUDGET = BN <= 64 ? 256 : 512;   // <= 256: two CTAs per SM
-  static constexpr int A_STAGES = STATIC ? 0 : (BN == 32 ? 2 : (BN == 64 ? 2 : 3));
+  // TMEM: a ring of bf16 A operands (weights, one 128 x 128 stage each) and
+  // the fp32 accumulator
+  // Two MMA-issuing threads (in different warps) each own half of every
+  // stage's k-steps and an accumulator of their own: one thread issues an
+  // MMA only every ~70 cycles, two issue in parallel.  The epilogue adds the
+  // two accumulators in a fixed order.
+  static constexpr int ISSUERS = 2;
+  static constexpr int A_STAGES = STATIC ? 0 : (BN == 64 ? 2 : 3);
   static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
-  static constexpr int NACC = BN == 16 ? 4 : (BN == 32 ? 4 : 2);
   static constexpr int ACC_COL = A_COLS;
-  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + NACC * BN);
-  static constexpr int RED_BYTES = BN * TILE_N * 4;        // split-K partial, reuses the stage buffers
-  static constexpr int BAR_BYTES = 8 * (2 * 6 + 2 * 6 + 3) + 16;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;   // + alignment slack
+  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + ISSUERS * BN);
+  static constexpr int RECV_OFF = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFF = RECV_OFF + RECV_BYTES;
+  static constexpr int BAR_BYTES = 8 * 40;
+  static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;   // + alignment slack
   static constexpr uint32_t IDESC = STATIC ? idesc_e4m3(BN) : idesc_bf16(BN);
-  static constexpr uint32_t TX_BYTES = CHUNK + X_BYTES;
-  static constexpr int THREADS = 320;
-  static_assert(A_COLS + NACC * BN <= TMEM_BUDGET, "TMEM budget");
-  static_assert(RED_BYTES <= STAGES * STAGE_BYTES, "split-K partial must fit the stage buffers");
+  static constexpr int THREADS = 352;   // producer, MMA issuer 0, 8 prologue warps, MMA issuer 1
+  static_assert(A_COLS + ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -199,36 +205,40 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
 }
 
 template <int FMT, int BN>
-__global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                                                          const GemmParams p) {
+__global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                                         const GemmParams p) {
   using C = GemmCfg<FMT, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);   // smem stage loaded
-  uint64_t* empty = full + C::STAGES;                                                // smem stage consumed
-  uint64_t* aready = empty + C::STAGES;   // operand ready: TMEM A slot (bf16) / shared e4m3 x (static)
-  uint64_t* aempty = aready + 6;          // TMEM A slot consumed
+  float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);
+  uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // stage's weight chunk landed
+  uint64_t* full_x = full_w + 6;          // stage's x tile landed
+  uint64_t* empty = full_x + 6;           // stage's shared memory consumed by the MMAs
+  uint64_t* aready = empty + 6;           // operand written: TMEM A slot (bf16) / shared e4m3 x (static)
+  uint64_t* aempty = aready + 6;          // TMEM A slot consumed by the MMAs
   uint64_t* acc_full = aempty + 6;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = acc_empty + 1;        // [2], one per MMA issuer
+  uint64_t* red_bar = drain + 2;          // split-K partials of every cluster CTA pushed here
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < 6; ++s) {
+      mbar_init(&full_w[s], 1);
+      mbar_init(&full_x[s], 1);
+      mbar_init(&empty[s], C::ISSUERS);
+      mbar_init(&aready[s], 8);
+      mbar_init(&aempty[s], C::ISSUERS);
     }
-    for (int a = 0; a < 6; ++a) {
-      mbar_init(&aready[a], 8);
-      mbar_init(&aempty[a], 1);
-    }
-    mbar_init(acc_full, 1);
+    mbar_init(acc_full, C::ISSUERS);
     mbar_init(acc_empty, 8);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    mbar_init(red_bar, 8 * (p.split > 1 ? p.split : 1));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -238,6 +248,9 @@ __global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // split-K: publish this CTA's barriers to the cluster now, wait for the
+  // peers' only right before pushing partials to them
+  if (p.split > 1) cluster_arrive_relaxed();
   pdl_launch_dependents();   // the next call may start its own prologue now
 
   const Work wk = cta_work(p);
@@ -247,78 +260,107 @@ __global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // (loop state is kept in counters: an integer division by a runtime
+      // value costs a long dependent chain on this latency-critical thread)
       const int total = wk.stages();
       const int pre = total < C::STAGES ? total : C::STAGES;
       // weights do not depend on earlier grids: stream the first stages now
-      for (int it = 0; it < pre; ++it) {
-        const int tile = wk.first_tile + (it / nst) * wk.tile_step, ks = wk.kb + it % nst;
-        mbar_arrive_expect_tx(&full[it], C::TX_BYTES);
-        bulk_g2s(smem + it * C::STAGE_BYTES + C::W_OFF,
-                 p.wchunks + ((size_t)(tile / p.m_tiles) * KS + ks) * C::CHUNK, C::CHUNK, &full[it]);
+      {
+        int ks = wk.kb, tile = wk.first_tile;
+        const uint8_t* wsrc = p.wchunks + (size_t)(tile / p.m_tiles) * KS * C::CHUNK;
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full_w[i], C::CHUNK);
+          bulk_g2s(smem + i * C::STAGE_BYTES + C::W_OFF, wsrc + (size_t)ks * C::CHUNK, C::CHUNK, &full_w[i]);
+          if (++ks == wk.ke) {
+            ks = wk.kb;
+            tile += wk.tile_step;
+            wsrc = p.wchunks + (size_t)(tile / p.m_tiles) * KS * C::CHUNK;
+          }
+        }
       }
       pdl_wait();   // x may be the previous grid's output
       bool ok = true;
-      int it = 0;
-      for (; ok && it < total; ++it) {
-        const int tile = wk.first_tile + (it / nst) * wk.tile_step, ks = wk.kb + it % nst;
-        const int m_tile = tile % p.m_tiles;
-        const int slot = it % C::STAGES;
-        uint8_t* st = smem + slot * C::STAGE_BYTES;
-        if (it >= pre) {
-          if (!mbar_wait(&empty[slot], ((it / C::STAGES) & 1) ^ 1, ctl)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[slot], C::TX_BYTES);
-          bulk_g2s(st + C::W_OFF, p.wchunks + ((size_t)(tile / p.m_tiles) * KS + ks) * C::CHUNK, C::CHUNK,
-                   &full[slot]);
+      int it = 0, slot = 0;
+      uint32_t ph = 0;
+      for (int t = 0; ok && t < wk.ntiles; ++t) {
+        const int tile = wk.first_tile + t * wk.tile_step;
+        const int n_tile = tile / p.m_tiles, m_tile = tile - n_tile * p.m_tiles;
+        const uint8_t* wsrc = p.wchunks + (size_t)n_tile * KS * C::CHUNK;
+        for (int ks = wk.kb; ks < wk.ke; ++ks, ++it) {
+          uint8_t* st = smem + slot * C::STAGE_BYTES;
+          if (it >= pre) {
+            if (!mbar_wait(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full_w[slot], C::CHUNK);
+            bulk_g2s(st + C::W_OFF, wsrc + (size_t)ks * C::CHUNK, C::CHUNK, &full_w[slot]);
+          }
+          mbar_arrive_expect_tx(&full_x[slot], C::X_BYTES);
+          if (p.x3d) {
+            tma_load_3d(st + C::X_OFF, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[slot]);
+          } else {
+            tma_load_2d(st + C::X_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[slot]);
+            tma_load_2d(st + C::X_OFF + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[slot]);
+          }
+          if (++slot == C::STAGES) {
+            slot = 0;
+            ph ^= 1;
+          }
         }
-        tma_load_2d(st + C::X_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full[slot]);
-        tma_load_2d(st + C::X_OFF + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full[slot]);
       }
       // Never leave with copies in flight: wait for the stages issued last
       // (a full barrier completes on data arrival alone; the loop only stops
-      // early after `pre`, so every prefetched stage got its x tile too).
+      // early after `pre`, so every issued stage has both its copies).
       volatile int no_abort = 0;
       const WaitCtl drain_ctl{&no_abort, p.status, p.timeout_ns};
-      const int issued = it > pre ? it : pre;
-      const int first = issued > C::STAGES ? issued - C::STAGES : 0;
-      for (int i = first; i < issued; ++i) mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
+      const int first = it > C::STAGES ? it - C::STAGES : 0;
+      for (int i = first; i < it; ++i) {
+        mbar_wait(&full_w[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
+        mbar_wait(&full_x[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
+      }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
-      int it = 0;
+      const int which = warp == 1 ? 0 : 1;   // k-steps [which*KK, (which+1)*KK) of each stage
+      constexpr int KK = C::STATIC ? 2 : 4;
+      const uint32_t d_tmem = tmem + C::ACC_COL + which * BN;
+      int it = 0, slot = 0, as = 0;
+      uint32_t ph = 0, aph = 0;
       bool ok = true;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
         if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl)) break;
         tc_fence_after();
         for (int j = 0; j < nst; ++j, ++it) {
-          const int slot = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait(&full[slot], ph, ctl)) { ok = false; break; }
           uint8_t* st = smem + slot * C::STAGE_BYTES;
           if constexpr (!C::STATIC) {
-            const int as = it % C::A_STAGES;
-            if (!mbar_wait(&aready[as], (it / C::A_STAGES) & 1, ctl)) { ok = false; break; }
+            if (!mbar_wait(&full_x[slot], ph, ctl) || !mbar_wait(&aready[as], aph, ctl)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t xb = smem_u32(st + C::X_OFF);
+            const uint32_t xb = smem_u32(st + C::X_OFF) + which * BN * 128;
+            const uint32_t a_tmem = tmem + as * (STAGE_K / 2) + which * KK * 8;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t bd = sdesc_sw128(xb + (kk >> 2) * BN * 128 + (kk & 3) * 32);
-              mma_bf16_ts(tmem + C::ACC_COL + (kk % C::NACC) * BN, tmem + as * (STAGE_K / 2) + kk * 8, bd,
-                          C::IDESC, (j > 0 || kk >= C::NACC) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < KK; ++kk)
+              mma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(xb + kk * 32), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&aempty[as]);
           } else {
-            if (!mbar_wait(&aready[slot], ph, ctl)) { ok = false; break; }
+            if (!mbar_wait(&full_w[slot], ph, ctl) || !mbar_wait(&aready[slot], ph, ctl)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t wb = smem_u32(st + C::W_OFF), qb = smem_u32(st + C::Q_OFF);
+            const uint32_t wb = smem_u32(st + C::W_OFF) + which * KK * 32, qb = smem_u32(st + C::Q_OFF) + which * KK * 32;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_f8_ss(tmem + C::ACC_COL + (kk % C::NACC) * BN, sdesc_sw128(wb + kk * 32),
-                        sdesc_sw128(qb + kk * 32), C::IDESC, (j > 0 || kk >= C::NACC) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < KK; ++kk)
+              mma_f8_ss(d_tmem, sdesc_sw128(wb + kk * 32), sdesc_sw128(qb + kk * 32), C::IDESC,
+                        (j > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&empty[slot]);
+          if (++slot == C::STAGES) {
+            slot = 0;
+            ph ^= 1;
+          }
+          if constexpr (!C::STATIC) {
+            if (++as == C::A_STAGES) {
+              as = 0;
+              aph ^= 1;
+            }
+          }
         }
         if (!ok) break;
         tc_commit(acc_full);
@@ -326,8 +368,8 @@ __global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // all MMAs this thread issued must finish before TMEM is released
       volatile int no_abort = 0;
       const WaitCtl drain_ctl{&no_abort, p.status, p.timeout_ns};
-      tc_commit(drain);
-      mbar_wait(drain, 0, drain_ctl);
+      tc_commit(&drain[which]);
+      mbar_wait(&drain[which], 0, drain_ctl);
     }
     __syncwarp();
   } else {
@@ -337,15 +379,30 @@ __global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     const int h = dw >> 2;              // k-half of the stage / column half of the tile
     const int r = qd * 32 + lane;       // weight row in the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+    constexpr int HALF = BN / 2;
+    float acc[HALF];
+    float e_sig = p.sigma, e_bias = 0.f;   // epilogue factor and bias of this thread's row
+    int n_row = 0, m_tile = 0;
     int it = 0;
-    bool ok = true;
+    bool ok = true, have_acc = false;
     for (int t = 0; ok && t < wk.ntiles; ++t) {
       const int tile = wk.first_tile + t * wk.tile_step;
+      m_tile = tile % p.m_tiles;
+      // this row's epilogue factor and bias: read-only, fetched now so the
+      // loads are long done when the epilogue needs them
+      n_row = (tile / p.m_tiles) * TILE_N + r;
+      e_sig = p.sigma;
+      e_bias = 0.f;
+      if (n_row < p.N) {
+        if (p.col_scale) e_sig = p.sigma * ld_nc_f32(p.col_scale + n_row);
+        if (p.bias) e_bias = ld_nc_bf16(p.bias + n_row);
+      }
       if constexpr (!C::STATIC) {
+        // the weight operand needs no x: the first A_STAGES stages are
+        // unpacked before the grid-dependency wait has even returned
         for (int j = 0; j < nst; ++j, ++it) {
           const int slot = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait_warp(&full[slot], ph, ctl)) { ok = false; break; }
+          if (!mbar_wait_warp(&full_w[slot], (it / C::STAGES) & 1, ctl)) { ok = false; break; }
           uint32_t o[32];
           prologue_stage<FMT, BN>(smem + slot * C::STAGE_BYTES + C::W_OFF, r, h, p.mx_bias, o);
           const int as = it % C::A_STAGES;
@@ -361,8 +418,8 @@ __global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         for (int j = 0; j < nst; ++j, ++it) {
           const int slot = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait_warp(&full[slot], ph, ctl)) { ok = false; break; }
-          // the shared B buffer of this slot is free once its previous MMAs finished
+          if (!mbar_wait_warp(&full_x[slot], ph, ctl)) { ok = false; break; }
+          // the shared e4m3 buffer of this slot is free once its previous MMAs finished
           if (!mbar_wait_warp(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
           uint8_t* st = smem + slot * C::STAGE_BYTES;
           quantize_x_tile<BN>(st + C::X_OFF, st + C::Q_OFF, p.s_x, threadIdx.x - 64);
@@ -376,83 +433,82 @@ __global__ void __launch_bounds__(320, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // ---- epilogue of this tile
       if (!mbar_wait_warp(acc_full, t & 1, ctl)) { ok = false; break; }
       tc_fence_after();
-      constexpr int HALF = BN / 2;
-      float acc[HALF];
 #pragma unroll
-      for (int a = 0; a < C::NACC; ++a) {
-        float v[HALF];
-#pragma unroll
-        for (int c8 = 0; c8 < HALF / 8; ++c8)
-          tmem_ld8(tmem + lane_base + C::ACC_COL + a * BN + h * HALF + c8 * 8,
-                   *reinterpret_cast<float(*)[8]>(v + c8 * 8));
+      for (int c8 = 0; c8 < HALF / 8; ++c8) {
+        float a1[8];
+        tmem_ld8(tmem + lane_base + C::ACC_COL + h * HALF + c8 * 8, *reinterpret_cast<float(*)[8]>(acc + c8 * 8));
+        tmem_ld8(tmem + lane_base + C::ACC_COL + BN + h * HALF + c8 * 8, a1);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < HALF; ++i) acc[i] = a == 0 ? v[i] : acc[i] + v[i];
+        for (int i = 0; i < 8; ++i) acc[c8 * 8 + i] += a1[i];
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
-      pdl_wait();   // y (and everything after) may be read by an earlier grid
+      have_acc = true;
       if (p.split == 1) {
-        const int n_tile = tile / p.m_tiles, m_tile = tile % p.m_tiles;
-        const int n = n_tile * TILE_N + r;
-        if (n < p.N) {
-          const float sig = p.col_scale ? p.sigma * p.col_scale[n] : p.sigma;
-          const float b = p.bias ? __bfloat162float(p.bias[n]) : 0.f;
+        pdl_wait();   // y may still be read by an earlier grid
+        if (n_row < p.N) {
 #pragma unroll
           for (int i = 0; i < HALF; ++i) {
             const int m = m_tile * BN + h * HALF + i;
-            if (m < p.M) p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(acc[i], sig, b));
+            if (m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(acc[i], e_sig, e_bias));
           }
         }
-      } else {
-        // split-K partial into this CTA's shared memory: [column][row]
-        float* red = reinterpret_cast<float*>(smem);
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) red[(h * HALF + i) * TILE_N + r] = acc[i];
       }
     }
     if (!ok) *abort_flag = 1;
-  }
 
-  if (p.split > 1) {
-    // ---- cluster split-K: every CTA of the cluster reaches both barriers
-    // (all 320 threads, whether or not their work completed)
-    __syncwarp();
-    cluster_sync();
-    if (warp >= 2 && !*abort_flag) {
+    if (p.split > 1) {
+      // ---- cluster split-K.  Rank q owns the tile's columns
+      // [q*BN/S, (q+1)*BN/S): every CTA stores its partial of those columns
+      // straight into the owner's shared memory and arrives on the owner's
+      // barrier; the owner sums the S partials of its columns in rank order.
+      // Every epilogue warp takes part (even after an abort) so that no CTA
+      // leaves while a peer may still write into it.
       const int S = p.split;
       const int q = (int)cluster_rank();
-      const int tile = blockIdx.x / S;
-      const int n_tile = tile / p.m_tiles, m_tile = tile % p.m_tiles;
-      // rank q finishes a slice of the tile's (column, row-quad) cells
-      const int cells = BN * (TILE_N / 4);
-      const int c0 = q * cells / S, c1 = (q + 1) * cells / S;
-      const float* red = reinterpret_cast<const float*>(smem);
-      for (int c = c0 + (int)threadIdx.x - 64; c < c1; c += 256) {
-        const int col = c / (TILE_N / 4), r4 = (c % (TILE_N / 4)) * 4;
-        float4 sum = ld_dsmem_f32x4(red + col * TILE_N + r4, 0);
-        for (int pr = 1; pr < S; ++pr) {
-          const float4 v = ld_dsmem_f32x4(red + col * TILE_N + r4, pr);
-          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-        }
-        const int m = m_tile * BN + col;
-        if (m < p.M) {
-          const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+      const int cmax = (BN + S - 1) / S;
+      const bool good = ok && have_acc;
+      pdl_wait();
+      cluster_wait();   // the peers' barriers are initialised
+      if (good) {
+        // this thread holds columns [h*HALF, (h+1)*HALF) of its row; walk
+        // them in order, moving to the next owner rank at each range end
+        int pr = ((h * HALF + 1) * S - 1) / BN;
+        int lo = pr * BN / S, hi = (pr + 1) * BN / S;
+        uint32_t base = dsmem_addr(recv + q * cmax * TILE_N + r, pr);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int n = n_tile * TILE_N + r4 + e;
-            if (n < p.N) {
-              const float sig = p.col_scale ? p.sigma * p.col_scale[n] : p.sigma;
-              const float b = p.bias ? __bfloat162float(p.bias[n]) : 0.f;
-              p.y[(size_t)m * p.N + n] = __float2bfloat16_rn(fmaf(vals[e], sig, b));
-            }
+        for (int i = 0; i < HALF; ++i) {
+          const int c = h * HALF + i;
+          if (c >= hi) {   // ranges hold >= 2 columns: one step is enough
+            ++pr;
+            lo = hi;
+            hi = (pr + 1) * BN / S;
+            base = dsmem_addr(recv + q * cmax * TILE_N + r, pr);
           }
+          st_dsmem_f32(base + (uint32_t)((c - lo) * TILE_N * 4), acc[i]);
+        }
+      }
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      __syncwarp();
+      if (lane == 0)
+        for (int pr = 0; pr < S; ++pr) mbar_arrive_remote(dsmem_addr(red_bar, pr));
+      // wait for every peer's push even after an abort: a peer may still be
+      // writing into this CTA's shared memory (bounded by the timeout alone)
+      volatile int no_abort = 0;
+      const WaitCtl red_ctl{&no_abort, p.status, p.timeout_ns};
+      const bool ok2 = mbar_wait_warp_cluster(red_bar, 0, red_ctl);
+      if (good && ok2 && !*abort_flag && n_row < p.N) {
+        const int c0 = q * BN / S, c1 = (q + 1) * BN / S;
+        for (int c = c0 + h; c < c1; c += 2) {
+          float sum = recv[((0 * cmax) + (c - c0)) * TILE_N + r];
+          for (int pr = 1; pr < S; ++pr) sum += recv[((pr * cmax) + (c - c0)) * TILE_N + r];
+          const int m = m_tile * BN + c;
+          if (m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
         }
       }
     }
-    __syncwarp();
-    cluster_sync();   // no CTA leaves while a peer may still read its partial
   }
 
   tc_fence_before();
