@@ -336,7 +336,8 @@ int cluster_capacity(dqgemm_s* h, int bn, int split) {
 // Tiles of 128 output channels x bn activation rows.  With at least one tile
 // per SM, each CTA computes whole tiles (persistent loop).  With fewer tiles
 // than SMs, the K range of each tile is split over the S CTAs of a cluster,
-// S the largest split (<= 8, <= k_stages) whose T * S CTAs are all resident.
+// S the largest power of two (<= 8, <= k_stages) whose T * S CTAs are all
+// resident.
 void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
   std::memset(pl, 0, sizeof(*pl));
   const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
@@ -356,13 +357,15 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
     const char* e = std::getenv("DQGEMM_SPLIT");
     return e ? std::atoi(e) : 0;
   }();
+  // the split is a power of two (<= 8, so it divides every bn): each rank
+  // then owns bn / S whole columns of the tile in the reduction
   int split = 1;
   if (force_split >= 1 && force_split <= 8) {
-    split = std::min(force_split, h->k_stages);
+    while (split * 2 <= std::min(force_split, h->k_stages)) split *= 2;
     if (split > 1 && cluster_capacity(h, bn, split) < T) split = 1;
   } else if (T < slots) {
-    for (int s = std::min(8, h->k_stages); s >= 2; --s) {
-      if (T * s > slots) continue;
+    for (int s = 8; s >= 2; s /= 2) {
+      if (s > h->k_stages || T * s > slots) continue;
       const int cap = cluster_capacity(h, bn, s);
       if (cap > 0 && cap >= T) { split = s; break; }
     }

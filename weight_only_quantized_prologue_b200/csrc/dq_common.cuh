@@ -58,11 +58,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Shared control block for bounded waits: every wait gives up after
-// `timeout_ns`, or as soon as another thread of the CTA has given up; the
+// Control of a bounded wait, passed by value (it lives in registers or is
+// rematerialised from kernel parameters; nothing of it goes to the stack):
+// every wait gives up after `timeout_ns`, or as soon as another thread of
+// the CTA has set the shared `abort` flag (null: ignore the flag); the
 // first thread to give up records DEV_TIMEOUT in the global status word.
 struct WaitCtl {
-  volatile int* abort;   // shared memory flag
+  volatile int* abort;   // shared memory flag, or null
   int* status;           // global status word (may be null)
   uint64_t timeout_ns;
 };
@@ -82,28 +84,32 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+__device__ __forceinline__ bool wait_give_up(const WaitCtl ctl, uint64_t t0) {
+  if (ctl.abort && *ctl.abort) return true;
+  if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+    if (ctl.abort) *ctl.abort = 1;
+    if (ctl.status) atomicExch(ctl.status, DEV_TIMEOUT);
+    return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
-    if (*ctl.abort) return false;
-    if (globaltimer_ns() - t0 > ctl.timeout_ns) {
-      *ctl.abort = 1;
-      if (ctl.status) atomicExch(ctl.status, DEV_TIMEOUT);
-      return false;
-    }
+    if (wait_give_up(ctl, t0)) return false;
   }
 }
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, ctl);
 }
 
 // Whole-warp wait: lane 0 sleeps on the barrier, the other lanes wait at the
-// warp barrier, then every lane re-tests the (now complete) phase so that each
-// thread has acquire ordering on the data the phase guards.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+// shuffle; then every lane observes the completed phase itself (acquire).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ctl) ? 1 : 0;
   ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -111,7 +117,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, c
   return ok != 0;
 }
 
-// wait with acquire at cluster scope (for data pushed by peer CTAs)
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -126,19 +131,14 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 
 // Whole-warp wait for data other CTAs of the cluster pushed into this CTA
 // (acquire at cluster scope); bounded like mbar_wait.
-__device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+__device__ __forceinline__ bool mbar_wait_cluster_slow(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*ctl.abort) return false;
-    if (globaltimer_ns() - t0 > ctl.timeout_ns) {
-      *ctl.abort = 1;
-      if (ctl.status) atomicExch(ctl.status, DEV_TIMEOUT);
-      return false;
-    }
+    if (wait_give_up(ctl, t0)) return false;
   }
 }
-__device__ __forceinline__ bool mbar_wait_warp_cluster(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+__device__ __forceinline__ bool mbar_wait_warp_cluster(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster_slow(bar, parity, ctl) ? 1 : 0;
   ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -243,6 +243,19 @@ __device__ __forceinline__ float4 ld_dsmem_f32x4(const void* local, uint32_t ran
                : "r"(remote)
                : "memory");
   return v;
+}
+
+// Bulk copy from this CTA's shared memory into another CTA of the cluster;
+// completes `bytes` of transaction count on the destination's mbarrier
+// (both given as shared::cluster addresses).  No multicast.
+__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// named barrier over a subset of the CTA's warps
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -63,10 +63,9 @@ struct GemmCfg {
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);
   static constexpr int W_OFF = Q_OFF + align_up(Q_BYTES, 1024);
   static constexpr int STAGE_BYTES = W_OFF + align_up(CHUNK, 1024);
-  // split-K receive buffer: partials pushed by the cluster's CTAs,
-  // [rank][column of this CTA's share (at most BN/2 + 1... bounded by BN/S+1)][row]
-  static constexpr int RECV_COLS = BN + 8;                 // >= S * ceil(BN / S) for S <= 8
-  static constexpr int RECV_BYTES = RECV_COLS * TILE_N * 4;
+  // split-K receive buffer: the S - 1 peers' partials of this CTA's BN / S
+  // columns, [peer slot][column][row] fp32 (S divides BN)
+  static constexpr int RECV_BYTES = BN * TILE_N * 4;
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
   static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : 200 * 1024;
@@ -219,12 +218,15 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint64_t* acc_full = aempty + 6;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;        // [2], one per MMA issuer
-  uint64_t* red_bar = drain + 2;          // split-K partials of every cluster CTA pushed here
+  uint64_t* red_bar = drain + 2;          // split-K: the peers' partials have landed in recv
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+  // wait control, rebuilt from kernel parameters at each wait so that it
+  // holds no registers across the long loops
+  const auto ctl = [&] { return WaitCtl{abort_flag, p.status, p.timeout_ns}; };
+  const auto ctl_no_abort = [&] { return WaitCtl{nullptr, p.status, p.timeout_ns}; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 6; ++s) {
@@ -238,7 +240,9 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     mbar_init(acc_empty, 8);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
-    mbar_init(red_bar, 8 * (p.split > 1 ? p.split : 1));
+    mbar_init(red_bar, 1);
+    // the peers' partials arrive as bulk copies counted in bytes
+    if (p.split > 1) mbar_arrive_expect_tx(red_bar, (uint32_t)((p.split - 1) * (BN / p.split) * TILE_N * 4));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         for (int ks = wk.kb; ks < wk.ke; ++ks, ++it) {
           uint8_t* st = smem + slot * C::STAGE_BYTES;
           if (it >= pre) {
-            if (!mbar_wait(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
+            if (!mbar_wait(&empty[slot], ph ^ 1, ctl())) { ok = false; break; }
             mbar_arrive_expect_tx(&full_w[slot], C::CHUNK);
             bulk_g2s(st + C::W_OFF, wsrc + (size_t)ks * C::CHUNK, C::CHUNK, &full_w[slot]);
           }
@@ -309,12 +313,10 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // Never leave with copies in flight: wait for the stages issued last
       // (a full barrier completes on data arrival alone; the loop only stops
       // early after `pre`, so every issued stage has both its copies).
-      volatile int no_abort = 0;
-      const WaitCtl drain_ctl{&no_abort, p.status, p.timeout_ns};
       const int first = it > C::STAGES ? it - C::STAGES : 0;
       for (int i = first; i < it; ++i) {
-        mbar_wait(&full_w[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
-        mbar_wait(&full_x[i % C::STAGES], (i / C::STAGES) & 1, drain_ctl);
+        mbar_wait(&full_w[i % C::STAGES], (i / C::STAGES) & 1, ctl_no_abort());
+        mbar_wait(&full_x[i % C::STAGES], (i / C::STAGES) & 1, ctl_no_abort());
       }
     }
     __syncwarp();
@@ -328,12 +330,12 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       uint32_t ph = 0, aph = 0;
       bool ok = true;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
-        if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl)) break;
+        if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl())) break;
         tc_fence_after();
         for (int j = 0; j < nst; ++j, ++it) {
           uint8_t* st = smem + slot * C::STAGE_BYTES;
           if constexpr (!C::STATIC) {
-            if (!mbar_wait(&full_x[slot], ph, ctl) || !mbar_wait(&aready[as], aph, ctl)) { ok = false; break; }
+            if (!mbar_wait(&full_x[slot], ph, ctl()) || !mbar_wait(&aready[as], aph, ctl())) { ok = false; break; }
             tc_fence_after();
             const uint32_t xb = smem_u32(st + C::X_OFF) + which * BN * 128;
             const uint32_t a_tmem = tmem + as * (STAGE_K / 2) + which * KK * 8;
@@ -342,7 +344,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
               mma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(xb + kk * 32), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&aempty[as]);
           } else {
-            if (!mbar_wait(&full_w[slot], ph, ctl) || !mbar_wait(&aready[slot], ph, ctl)) { ok = false; break; }
+            if (!mbar_wait(&full_w[slot], ph, ctl()) || !mbar_wait(&aready[slot], ph, ctl())) { ok = false; break; }
             tc_fence_after();
             const uint32_t wb = smem_u32(st + C::W_OFF) + which * KK * 32, qb = smem_u32(st + C::Q_OFF) + which * KK * 32;
 #pragma unroll
@@ -366,10 +368,8 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         tc_commit(acc_full);
       }
       // all MMAs this thread issued must finish before TMEM is released
-      volatile int no_abort = 0;
-      const WaitCtl drain_ctl{&no_abort, p.status, p.timeout_ns};
       tc_commit(&drain[which]);
-      mbar_wait(&drain[which], 0, drain_ctl);
+      mbar_wait(&drain[which], 0, ctl_no_abort());
     }
     __syncwarp();
   } else {
@@ -402,11 +402,11 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         // unpacked before the grid-dependency wait has even returned
         for (int j = 0; j < nst; ++j, ++it) {
           const int slot = it % C::STAGES;
-          if (!mbar_wait_warp(&full_w[slot], (it / C::STAGES) & 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_warp(&full_w[slot], (it / C::STAGES) & 1, ctl())) { ok = false; break; }
           uint32_t o[32];
           prologue_stage<FMT, BN>(smem + slot * C::STAGE_BYTES + C::W_OFF, r, h, p.mx_bias, o);
           const int as = it % C::A_STAGES;
-          if (!mbar_wait_warp(&aempty[as], ((it / C::A_STAGES) & 1) ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_warp(&aempty[as], ((it / C::A_STAGES) & 1) ^ 1, ctl())) { ok = false; break; }
           tc_fence_after();
           tmem_st32(tmem + lane_base + as * (STAGE_K / 2) + h * 32, o);
           tmem_wait_st();
@@ -418,9 +418,9 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         for (int j = 0; j < nst; ++j, ++it) {
           const int slot = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait_warp(&full_x[slot], ph, ctl)) { ok = false; break; }
+          if (!mbar_wait_warp(&full_x[slot], ph, ctl())) { ok = false; break; }
           // the shared e4m3 buffer of this slot is free once its previous MMAs finished
-          if (!mbar_wait_warp(&empty[slot], ph ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_warp(&empty[slot], ph ^ 1, ctl())) { ok = false; break; }
           uint8_t* st = smem + slot * C::STAGE_BYTES;
           quantize_x_tile<BN>(st + C::X_OFF, st + C::Q_OFF, p.s_x, threadIdx.x - 64);
           fence_proxy_async_smem();
@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       if (!ok) break;
 
       // ---- epilogue of this tile
-      if (!mbar_wait_warp(acc_full, t & 1, ctl)) { ok = false; break; }
+      if (!mbar_wait_warp(acc_full, t & 1, ctl())) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int c8 = 0; c8 < HALF / 8; ++c8) {
@@ -446,8 +446,9 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       have_acc = true;
+      // (no grid-dependency wait here: the producer's wait precedes the x
+      // loads this accumulator depends on, so every earlier grid is done)
       if (p.split == 1) {
-        pdl_wait();   // y may still be read by an earlier grid
         if (n_row < p.N) {
 #pragma unroll
           for (int i = 0; i < HALF; ++i) {
@@ -461,49 +462,44 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
 
     if (p.split > 1) {
       // ---- cluster split-K.  Rank q owns the tile's columns
-      // [q*BN/S, (q+1)*BN/S): every CTA stores its partial of those columns
-      // straight into the owner's shared memory and arrives on the owner's
-      // barrier; the owner sums the S partials of its columns in rank order.
-      // Every epilogue warp takes part (even after an abort) so that no CTA
-      // leaves while a peer may still write into it.
+      // [q*BN/S, (q+1)*BN/S).  Each CTA writes its whole partial tile into
+      // its own (now idle) stage buffers as [column][row] fp32, then one
+      // thread sends every peer the block of that peer's columns with one
+      // bulk copy that completes on the peer's red_bar.  The owner adds the
+      // S partials of its columns in rank order (deterministic).  Every
+      // epilogue warp takes part even after an abort.
       const int S = p.split;
       const int q = (int)cluster_rank();
-      const int cmax = (BN + S - 1) / S;
+      const int cmax = BN / S;
       const bool good = ok && have_acc;
-      pdl_wait();
-      cluster_wait();   // the peers' barriers are initialised
+      float* part = reinterpret_cast<float*>(smem);   // [BN][TILE_N]; all MMAs are done
       if (good) {
-        // this thread holds columns [h*HALF, (h+1)*HALF) of its row; walk
-        // them in order, moving to the next owner rank at each range end
-        int pr = ((h * HALF + 1) * S - 1) / BN;
-        int lo = pr * BN / S, hi = (pr + 1) * BN / S;
-        uint32_t base = dsmem_addr(recv + q * cmax * TILE_N + r, pr);
 #pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const int c = h * HALF + i;
-          if (c >= hi) {   // ranges hold >= 2 columns: one step is enough
-            ++pr;
-            lo = hi;
-            hi = (pr + 1) * BN / S;
-            base = dsmem_addr(recv + q * cmax * TILE_N + r, pr);
-          }
-          st_dsmem_f32(base + (uint32_t)((c - lo) * TILE_N * 4), acc[i]);
+        for (int i = 0; i < HALF; ++i) part[(h * HALF + i) * TILE_N + r] = acc[i];
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 256);
+      cluster_wait();   // the peers' barriers are initialised and armed
+      if (threadIdx.x == 64) {
+        for (int pr = 0; pr < S; ++pr) {
+          if (pr == q) continue;
+          const int slot = q < pr ? q : q - 1;   // this CTA's slot in the peer's recv
+          bulk_s2cluster(dsmem_addr(recv + slot * cmax * TILE_N, pr), part + pr * cmax * TILE_N,
+                         (uint32_t)(cmax * TILE_N * 4), dsmem_addr(red_bar, pr));
         }
       }
-      asm volatile("fence.acq_rel.cluster;" ::: "memory");
-      __syncwarp();
-      if (lane == 0)
-        for (int pr = 0; pr < S; ++pr) mbar_arrive_remote(dsmem_addr(red_bar, pr));
-      // wait for every peer's push even after an abort: a peer may still be
-      // writing into this CTA's shared memory (bounded by the timeout alone)
-      volatile int no_abort = 0;
-      const WaitCtl red_ctl{&no_abort, p.status, p.timeout_ns};
-      const bool ok2 = mbar_wait_warp_cluster(red_bar, 0, red_ctl);
+      // wait for every peer's partial even after an abort (bounded by the
+      // timeout alone)
+      const bool ok2 = mbar_wait_warp_cluster(red_bar, 0, ctl_no_abort());
       if (good && ok2 && !*abort_flag && n_row < p.N) {
-        const int c0 = q * BN / S, c1 = (q + 1) * BN / S;
-        for (int c = c0 + h; c < c1; c += 2) {
-          float sum = recv[((0 * cmax) + (c - c0)) * TILE_N + r];
-          for (int pr = 1; pr < S; ++pr) sum += recv[((pr * cmax) + (c - c0)) * TILE_N + r];
+        const int c0 = q * cmax;
+        for (int c = c0 + h; c < c0 + cmax; c += 2) {
+          float sum = 0.f;
+          for (int pr = 0; pr < S; ++pr) {
+            const float v = pr == q ? part[c * TILE_N + r]
+                                    : recv[((pr < q ? pr : pr - 1) * cmax + (c - c0)) * TILE_N + r];
+            sum = pr == 0 ? v : sum + v;
+          }
           const int m = m_tile * BN + c;
           if (m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
         }
@@ -511,6 +507,14 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     }
   }
 
+  __syncwarp();
+  if (p.split > 1) {
+    // no CTA leaves while a copy out of or into its shared memory may be in
+    // flight: every CTA arrives here only after all its incoming partials
+    // landed, so once all have arrived every copy of the cluster is done
+    if (warp < 2 || warp == 10) cluster_wait();   // the epilogue warps waited above
+    cluster_sync();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
