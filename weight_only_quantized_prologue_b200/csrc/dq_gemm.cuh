@@ -5,17 +5,19 @@
 // rows are its N (BN = 16..128): the skinny decode shapes the quantized-Linear
 // pages run (x of 32 rows) keep the tensor core busy on the weight side.
 //
-// CTA = 10 warps, warp-specialized:
+// CTA = 11 warps, warp-specialized:
 //   warp 0      producer: one 1-D bulk copy of the stage's pre-tiled weight
-//               chunk + two TMA box loads of the bf16 x tile, per stage
-//   warp 1      MMA issuer: one thread issues tcgen05.mma into a TMEM
-//               accumulator and commits stage / operand / accumulator barriers
+//               chunk + the TMA box load(s) of the bf16 x tile, per stage
+//   warps 1, 10 MMA issuers: one thread each issues tcgen05.mma for half of
+//               every stage's k-steps into its own TMEM accumulator (a single
+//               thread issues only one MMA every ~80 cycles) and commits the
+//               stage / operand / accumulator barriers
 //   warps 2..9  the prologue: unpack + scale the packed codes of one weight
 //               row per thread (two threads per row, one per k-half) into
 //               bf16 operands written straight to TMEM (the MMA reads A from
 //               TMEM), or, for static FP8, quantize the x tile to e4m3 into
-//               shared memory; then the epilogue (tcgen05.ld, scale, bias,
-//               bf16 cast, store).
+//               shared memory; then the epilogue (tcgen05.ld of both
+//               accumulators, scale, bias, bf16 cast, store).
 // Work split: a tile of 128 output channels x BN activation rows is either
 // computed whole by one CTA (persistent loop over tiles), or its K range is
 // split over the S CTAs of a thread-block cluster whose fp32 partials are
@@ -59,37 +61,51 @@ struct GemmCfg {
   static constexpr int CHUNK = chunk_bytes(FMT);
   static constexpr int X_BYTES = BN * 256;                 // two 64-k blocks of BN rows x 128 B
   static constexpr int Q_BYTES = STATIC ? BN * 128 : 0;    // e4m3 x tile (static FP8)
-  static constexpr int X_OFF = 0;
-  static constexpr int Q_OFF = align_up(X_BYTES, 1024);
-  static constexpr int W_OFF = Q_OFF + align_up(Q_BYTES, 1024);
-  static constexpr int STAGE_BYTES = W_OFF + align_up(CHUNK, 1024);
+  // Two rings: packed weight chunks (streamed from the start of the kernel;
+  // a slot is free once the prologue has read it, or for static FP8 once the
+  // MMAs have) and x tiles (loaded only after the grid-dependency wait; a
+  // slot is free once the MMAs have read it).
+  static constexpr int X_SLOT = align_up(X_BYTES, 1024) + align_up(Q_BYTES, 1024);
+  static constexpr int Q_OFF = align_up(X_BYTES, 1024);    // within an x slot
+  static constexpr int W_SLOT = align_up(CHUNK, 1024);
+  static constexpr int XST = BN <= 32 ? 3 : 2;
   // split-K receive buffer: the S - 1 peers' partials of this CTA's BN / S
   // columns, [peer slot][column][row] fp32 (S divides BN)
   static constexpr int RECV_BYTES = BN * TILE_N * 4;
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
   static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : 200 * 1024;
-  static constexpr int STAGES_RAW = (SMEM_BUDGET - RECV_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW < 2 ? 2 : (STAGES_RAW > 6 ? 6 : STAGES_RAW);
+  static constexpr int WST_RAW = (SMEM_BUDGET - XST * X_SLOT - RECV_BYTES - 3072) / W_SLOT;   // barriers, EPI, slack
+  static constexpr int WST = WST_RAW < 2 ? 2 : (WST_RAW > 8 ? 8 : WST_RAW);
+  static constexpr int STAGES = WST;   // weight stages in flight (reported by the plan)
+  static constexpr int X_RING_OFF = 0;
+  static constexpr int W_RING_OFF = XST * X_SLOT;
   // TMEM: a ring of bf16 A operands (weights, one 128 x 128 stage each) and
-  // the fp32 accumulator
-  // Two MMA-issuing threads (in different warps) each own half of every
-  // stage's k-steps and an accumulator of their own: one thread issues an
-  // MMA only every ~70 cycles, two issue in parallel.  The epilogue adds the
-  // two accumulators in a fixed order.
+  // the fp32 accumulators.  Two MMA-issuing threads (in different warps) each
+  // own half of every stage's k-steps and an accumulator of their own: one
+  // thread issues an MMA only every ~80 cycles, two issue in parallel.  The
+  // epilogue adds the two accumulators in a fixed order.
   static constexpr int ISSUERS = 2;
   static constexpr int A_STAGES = STATIC ? 0 : (BN == 64 ? 2 : 3);
   static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
   static constexpr int TMEM_COLS = pow2_at_least(A_COLS + ISSUERS * BN);
-  static constexpr int RECV_OFF = STAGES * STAGE_BYTES;
+  static constexpr int RECV_OFF = W_RING_OFF + WST * W_SLOT;
   static constexpr int BAR_OFF = RECV_OFF + RECV_BYTES;
   static constexpr int BAR_BYTES = 8 * 40;
-  static constexpr int SMEM = BAR_OFF + BAR_BYTES + 1024;   // + alignment slack
+  // each epilogue thread's row factor and bias, parked in shared memory over
+  // the main loop instead of holding registers: [2][256] fp32
+  static constexpr int EPI_OFF = BAR_OFF + BAR_BYTES;
+  static constexpr int EPI_BYTES = 2 * 256 * 4;
+  static constexpr int SMEM = EPI_OFF + EPI_BYTES + 1024;   // + alignment slack
   static constexpr uint32_t IDESC = STATIC ? idesc_e4m3(BN) : idesc_bf16(BN);
-  static constexpr int THREADS = 352;   // producer, MMA issuer 0, 8 prologue warps, MMA issuer 1
+  // warp 0 weight producer, 1 and 10 MMA issuers, 2..9 prologue/epilogue,
+  // 11 x producer
+  static constexpr int THREADS = 384;
   static_assert(A_COLS + ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
-  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");   // (two CTAs per SM need <= 113 KB)
+  static_assert(A_STAGES <= 3 && XST <= 3, "barrier arrays");
+  static_assert(XST * X_SLOT >= BN * TILE_N * 4, "split-K partial tile fits in the x ring");
 };
 
 // The work of one CTA: a list of (tile, k_begin, k_end) segments.
@@ -118,62 +134,56 @@ __device__ __forceinline__ Work cta_work(const GemmParams& p) {
   return w;
 }
 
-template <int FMT, int BN>
-__device__ __forceinline__ void prologue_stage(const uint8_t* chunk, int r, int h, int mx_bias, uint32_t (&o)[32]) {
+// One half (hp = 0: k-steps 0..3, hp = 1: 4..7 of this thread's k-half) of
+// the operand a prologue thread produces per stage: 16 words of bf16x2 for
+// weight row r, in TMEM column order.  Working in halves keeps the live
+// registers of the unpack low.
+template <int FMT>
+__device__ __forceinline__ void prologue_half(const uint8_t* chunk, int r, int h, int hp, int mx_bias, uint32_t (&o)[16]) {
   if constexpr (FMT == FMT_FP8) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 v = lds128(chunk + ((h * 4 + j) * TILE_N + r) * 16);
+    for (int j = 0; j < 2; ++j) {
+      const uint4 v = lds128(chunk + ((h * 4 + hp * 2 + j) * TILE_N + r) * 16);
       unpack_e4m3(v.x, o + j * 8 + 0);
       unpack_e4m3(v.y, o + j * 8 + 2);
       unpack_e4m3(v.z, o + j * 8 + 4);
       unpack_e4m3(v.w, o + j * 8 + 6);
     }
   } else {
-    const uint4 v0 = lds128(chunk + ((h * 2 + 0) * TILE_N + r) * 16);
-    const uint4 v1 = lds128(chunk + ((h * 2 + 1) * TILE_N + r) * 16);
+    const uint4 v = lds128(chunk + ((h * 2 + hp) * TILE_N + r) * 16);
     const uint8_t* sc = chunk + PACKED4_BYTES;
+    uint32_t sa, sb;   // bf16x2 scale words of the two 8-word halves of v
     if constexpr (FMT == FMT_INT4) {
       const uint32_t s = *reinterpret_cast<const uint16_t*>(sc + r * 2);
-      const uint32_t s2 = s | (s << 16);
-      unpack_int4(v0.x, s2, o + 0);
-      unpack_int4(v0.y, s2, o + 4);
-      unpack_int4(v0.z, s2, o + 8);
-      unpack_int4(v0.w, s2, o + 12);
-      unpack_int4(v1.x, s2, o + 16);
-      unpack_int4(v1.y, s2, o + 20);
-      unpack_int4(v1.z, s2, o + 24);
-      unpack_int4(v1.w, s2, o + 28);
+      sa = sb = s | (s << 16);
     } else if constexpr (FMT == FMT_NVFP4) {
-      const uint32_t c4 = *reinterpret_cast<const uint32_t*>(sc + (h * TILE_N + r) * 4);
-      uint32_t s2[4];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t s = nvfp4_scale_bf16((c4 >> (8 * b)) & 0xFFu);
-        s2[b] = s | (s << 16);
-      }
-      unpack_e2m1(v0.x, s2[0], o + 0);
-      unpack_e2m1(v0.y, s2[0], o + 4);
-      unpack_e2m1(v0.z, s2[1], o + 8);
-      unpack_e2m1(v0.w, s2[1], o + 12);
-      unpack_e2m1(v1.x, s2[2], o + 16);
-      unpack_e2m1(v1.y, s2[2], o + 20);
-      unpack_e2m1(v1.z, s2[3], o + 24);
-      unpack_e2m1(v1.w, s2[3], o + 28);
-    } else {  // MXFP4
-      const uint32_t c2 = *reinterpret_cast<const uint16_t*>(sc + (h * TILE_N + r) * 2);
-      const uint32_t sa = mxfp4_scale_bf16(c2 & 0xFFu, mx_bias), sb = mxfp4_scale_bf16(c2 >> 8, mx_bias);
-      const uint32_t s2a = sa | (sa << 16), s2b = sb | (sb << 16);
-      unpack_e2m1(v0.x, s2a, o + 0);
-      unpack_e2m1(v0.y, s2a, o + 4);
-      unpack_e2m1(v0.z, s2a, o + 8);
-      unpack_e2m1(v0.w, s2a, o + 12);
-      unpack_e2m1(v1.x, s2b, o + 16);
-      unpack_e2m1(v1.y, s2b, o + 20);
-      unpack_e2m1(v1.z, s2b, o + 24);
-      unpack_e2m1(v1.w, s2b, o + 28);
+      const uint32_t c2 = *reinterpret_cast<const uint16_t*>(sc + (h * TILE_N + r) * 4 + hp * 2);
+      const uint32_t a = nvfp4_scale_bf16(c2 & 0xFFu), b = nvfp4_scale_bf16(c2 >> 8);
+      sa = a | (a << 16);
+      sb = b | (b << 16);
+    } else {  // MXFP4: one scale per 32 = per half
+      const uint32_t c = *(sc + (h * TILE_N + r) * 2 + hp);
+      const uint32_t a = mxfp4_scale_bf16(c, mx_bias);
+      sa = sb = a | (a << 16);
+    }
+    if constexpr (FMT == FMT_INT4) {
+      unpack_int4(v.x, sa, o + 0);
+      unpack_int4(v.y, sa, o + 4);
+      unpack_int4(v.z, sb, o + 8);
+      unpack_int4(v.w, sb, o + 12);
+    } else {
+      unpack_e2m1(v.x, sa, o + 0);
+      unpack_e2m1(v.y, sa, o + 4);
+      unpack_e2m1(v.z, sb, o + 8);
+      unpack_e2m1(v.w, sb, o + 12);
     }
   }
+}
+
+template <int FMT, int BN>
+__device__ __forceinline__ void prologue_stage(const uint8_t* chunk, int r, int h, int mx_bias, uint32_t (&o)[32]) {
+  prologue_half<FMT>(chunk, r, h, 0, mx_bias, *reinterpret_cast<uint32_t(*)[16]>(o));
+  prologue_half<FMT>(chunk, r, h, 1, mx_bias, *reinterpret_cast<uint32_t(*)[16]>(o + 16));
 }
 
 // Static FP8: quantize the bf16 x tile (two SW128 boxes) into the e4m3 SW128
@@ -204,18 +214,21 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
 }
 
 template <int FMT, int BN>
-__global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
+__global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                          const GemmParams p) {
   using C = GemmCfg<FMT, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* x_ring = smem + C::X_RING_OFF;
+  uint8_t* w_ring = smem + C::W_RING_OFF;
   float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);
-  uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // stage's weight chunk landed
-  uint64_t* full_x = full_w + 6;          // stage's x tile landed
-  uint64_t* empty = full_x + 6;           // stage's shared memory consumed by the MMAs
-  uint64_t* aready = empty + 6;           // operand written: TMEM A slot (bf16) / shared e4m3 x (static)
-  uint64_t* aempty = aready + 6;          // TMEM A slot consumed by the MMAs
-  uint64_t* acc_full = aempty + 6;
+  uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [8] weight chunk landed
+  uint64_t* wempty = full_w + 8;          // [8] weight slot read (prologue, or MMAs for static FP8)
+  uint64_t* full_x = wempty + 8;          // [3] x tile landed
+  uint64_t* xempty = full_x + 3;          // [3] x slot read by the MMAs
+  uint64_t* aready = xempty + 3;          // [3] operand written: TMEM A slot (bf16) / e4m3 x (static, per x slot)
+  uint64_t* aempty = aready + 3;          // [3] TMEM A slot read by the MMAs
+  uint64_t* acc_full = aempty + 3;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;        // [2], one per MMA issuer
   uint64_t* red_bar = drain + 2;          // split-K: the peers' partials have landed in recv
@@ -229,10 +242,13 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   const auto ctl_no_abort = [&] { return WaitCtl{nullptr, p.status, p.timeout_ns}; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 6; ++s) {
+    for (int s = 0; s < 8; ++s) {
       mbar_init(&full_w[s], 1);
+      mbar_init(&wempty[s], C::STATIC ? C::ISSUERS : 8);
+    }
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&full_x[s], 1);
-      mbar_init(&empty[s], C::ISSUERS);
+      mbar_init(&xempty[s], C::ISSUERS);
       mbar_init(&aready[s], 8);
       mbar_init(&aempty[s], C::ISSUERS);
     }
@@ -247,7 +263,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_slot, C::TMEM_COLS);
-  if (warp == 1 && lane == 0) prefetch_tmap(&tmap_x);
+  if (warp == 11 && lane == 0) prefetch_tmap(&tmap_x);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -260,64 +276,65 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   const Work wk = cta_work(p);
   const int KS = p.k_stages;
   const int nst = wk.ke - wk.kb;   // stages per tile
+  // (all ring positions are kept in counters: an integer division by a
+  // runtime value costs a long dependent chain on the single-thread roles)
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ weight producer
+    // Weights do not depend on earlier grids: they stream from the start, as
+    // far ahead as the ring allows.
     if (lane == 0) {
-      // (loop state is kept in counters: an integer division by a runtime
-      // value costs a long dependent chain on this latency-critical thread)
       const int total = wk.stages();
-      const int pre = total < C::STAGES ? total : C::STAGES;
-      // weights do not depend on earlier grids: stream the first stages now
-      {
-        int ks = wk.kb, tile = wk.first_tile;
-        const uint8_t* wsrc = p.wchunks + (size_t)(tile / p.m_tiles) * KS * C::CHUNK;
-        for (int i = 0; i < pre; ++i) {
-          mbar_arrive_expect_tx(&full_w[i], C::CHUNK);
-          bulk_g2s(smem + i * C::STAGE_BYTES + C::W_OFF, wsrc + (size_t)ks * C::CHUNK, C::CHUNK, &full_w[i]);
-          if (++ks == wk.ke) {
-            ks = wk.kb;
-            tile += wk.tile_step;
-            wsrc = p.wchunks + (size_t)(tile / p.m_tiles) * KS * C::CHUNK;
-          }
+      int ks = wk.kb, tile = wk.first_tile, ws = 0, it = 0;
+      uint32_t wph = 0;
+      const uint8_t* wsrc = p.wchunks + (size_t)(tile / p.m_tiles) * KS * C::CHUNK;
+      for (; it < total; ++it) {
+        if (it >= C::WST && !mbar_wait(&wempty[ws], wph ^ 1, ctl())) break;
+        mbar_arrive_expect_tx(&full_w[ws], C::CHUNK);
+        bulk_g2s(w_ring + ws * C::W_SLOT, wsrc + (size_t)ks * C::CHUNK, C::CHUNK, &full_w[ws]);
+        if (++ks == wk.ke) {
+          ks = wk.kb;
+          tile += wk.tile_step;
+          wsrc = p.wchunks + (size_t)(tile / p.m_tiles) * KS * C::CHUNK;
+        }
+        if (++ws == C::WST) {
+          ws = 0;
+          wph ^= 1;
         }
       }
+      // never leave with copies in flight: wait for the chunks issued last
+      for (int i = it > C::WST ? it - C::WST : 0; i < it; ++i)
+        mbar_wait(&full_w[i % C::WST], (i / C::WST) & 1, ctl_no_abort());
+    }
+    __syncwarp();
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ x producer
+    if (lane == 0) {
       pdl_wait();   // x may be the previous grid's output
+      int xs = 0, it = 0;
+      uint32_t xph = 0;
       bool ok = true;
-      int it = 0, slot = 0;
-      uint32_t ph = 0;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
         const int tile = wk.first_tile + t * wk.tile_step;
-        const int n_tile = tile / p.m_tiles, m_tile = tile - n_tile * p.m_tiles;
-        const uint8_t* wsrc = p.wchunks + (size_t)n_tile * KS * C::CHUNK;
+        const int m_tile = tile - (tile / p.m_tiles) * p.m_tiles;
         for (int ks = wk.kb; ks < wk.ke; ++ks, ++it) {
-          uint8_t* st = smem + slot * C::STAGE_BYTES;
-          if (it >= pre) {
-            if (!mbar_wait(&empty[slot], ph ^ 1, ctl())) { ok = false; break; }
-            mbar_arrive_expect_tx(&full_w[slot], C::CHUNK);
-            bulk_g2s(st + C::W_OFF, wsrc + (size_t)ks * C::CHUNK, C::CHUNK, &full_w[slot]);
-          }
-          mbar_arrive_expect_tx(&full_x[slot], C::X_BYTES);
+          if (it >= C::XST && !mbar_wait(&xempty[xs], xph ^ 1, ctl())) { ok = false; break; }
+          uint8_t* xd = x_ring + xs * C::X_SLOT;
+          mbar_arrive_expect_tx(&full_x[xs], C::X_BYTES);
           if (p.x3d) {
-            tma_load_3d(st + C::X_OFF, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[slot]);
+            tma_load_3d(xd, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[xs]);
           } else {
-            tma_load_2d(st + C::X_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[slot]);
-            tma_load_2d(st + C::X_OFF + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[slot]);
+            tma_load_2d(xd, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
+            tma_load_2d(xd + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[xs]);
           }
-          if (++slot == C::STAGES) {
-            slot = 0;
-            ph ^= 1;
+          if (++xs == C::XST) {
+            xs = 0;
+            xph ^= 1;
           }
         }
       }
-      // Never leave with copies in flight: wait for the stages issued last
-      // (a full barrier completes on data arrival alone; the loop only stops
-      // early after `pre`, so every issued stage has both its copies).
-      const int first = it > C::STAGES ? it - C::STAGES : 0;
-      for (int i = first; i < it; ++i) {
-        mbar_wait(&full_w[i % C::STAGES], (i / C::STAGES) & 1, ctl_no_abort());
-        mbar_wait(&full_x[i % C::STAGES], (i / C::STAGES) & 1, ctl_no_abort());
-      }
+      for (int i = it > C::XST ? it - C::XST : 0; i < it; ++i)
+        mbar_wait(&full_x[i % C::XST], (i / C::XST) & 1, ctl_no_abort());
     }
     __syncwarp();
   } else if (warp == 1 || warp == 10) {
@@ -326,42 +343,46 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       const int which = warp == 1 ? 0 : 1;   // k-steps [which*KK, (which+1)*KK) of each stage
       constexpr int KK = C::STATIC ? 2 : 4;
       const uint32_t d_tmem = tmem + C::ACC_COL + which * BN;
-      int it = 0, slot = 0, as = 0;
-      uint32_t ph = 0, aph = 0;
+      int ws = 0, xs = 0, as = 0;
+      uint32_t wph = 0, xph = 0, aph = 0;
       bool ok = true;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
         if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl())) break;
         tc_fence_after();
-        for (int j = 0; j < nst; ++j, ++it) {
-          uint8_t* st = smem + slot * C::STAGE_BYTES;
+        for (int j = 0; j < nst; ++j) {
+          const uint32_t xb = smem_u32(x_ring + xs * C::X_SLOT);
           if constexpr (!C::STATIC) {
-            if (!mbar_wait(&full_x[slot], ph, ctl()) || !mbar_wait(&aready[as], aph, ctl())) { ok = false; break; }
+            if (!mbar_wait(&full_x[xs], xph, ctl()) || !mbar_wait(&aready[as], aph, ctl())) { ok = false; break; }
             tc_fence_after();
-            const uint32_t xb = smem_u32(st + C::X_OFF) + which * BN * 128;
+            const uint32_t bx = xb + which * BN * 128;
             const uint32_t a_tmem = tmem + as * (STAGE_K / 2) + which * KK * 8;
 #pragma unroll
             for (int kk = 0; kk < KK; ++kk)
-              mma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(xb + kk * 32), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
+              mma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(bx + kk * 32), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&aempty[as]);
-          } else {
-            if (!mbar_wait(&full_w[slot], ph, ctl()) || !mbar_wait(&aready[slot], ph, ctl())) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t wb = smem_u32(st + C::W_OFF) + which * KK * 32, qb = smem_u32(st + C::Q_OFF) + which * KK * 32;
-#pragma unroll
-            for (int kk = 0; kk < KK; ++kk)
-              mma_f8_ss(d_tmem, sdesc_sw128(wb + kk * 32), sdesc_sw128(qb + kk * 32), C::IDESC,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(&empty[slot]);
-          if (++slot == C::STAGES) {
-            slot = 0;
-            ph ^= 1;
-          }
-          if constexpr (!C::STATIC) {
             if (++as == C::A_STAGES) {
               as = 0;
               aph ^= 1;
             }
+          } else {
+            if (!mbar_wait(&full_w[ws], wph, ctl()) || !mbar_wait(&aready[xs], xph, ctl())) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t wb = smem_u32(w_ring + ws * C::W_SLOT) + which * KK * 32;
+            const uint32_t qb = xb + C::Q_OFF + which * KK * 32;
+#pragma unroll
+            for (int kk = 0; kk < KK; ++kk)
+              mma_f8_ss(d_tmem, sdesc_sw128(wb + kk * 32), sdesc_sw128(qb + kk * 32), C::IDESC,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&wempty[ws]);
+            if (++ws == C::WST) {
+              ws = 0;
+              wph ^= 1;
+            }
+          }
+          tc_commit(&xempty[xs]);
+          if (++xs == C::XST) {
+            xs = 0;
+            xph ^= 1;
           }
         }
         if (!ok) break;
@@ -381,55 +402,75 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
     constexpr int HALF = BN / 2;
     float acc[HALF];
-    float e_sig = p.sigma, e_bias = 0.f;   // epilogue factor and bias of this thread's row
-    int n_row = 0, m_tile = 0;
-    int it = 0;
+    float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);   // [2][256]: this thread's slots only
+    const int et = threadIdx.x - 64;
+    int tile = 0;
+    int ws = 0, xs = 0, as = 0;
+    uint32_t wph = 0, xph = 0, aph = 0;
     bool ok = true, have_acc = false;
     for (int t = 0; ok && t < wk.ntiles; ++t) {
-      const int tile = wk.first_tile + t * wk.tile_step;
-      m_tile = tile % p.m_tiles;
+      tile = wk.first_tile + t * wk.tile_step;
       // this row's epilogue factor and bias: read-only, fetched now so the
       // loads are long done when the epilogue needs them
-      n_row = (tile / p.m_tiles) * TILE_N + r;
-      e_sig = p.sigma;
-      e_bias = 0.f;
-      if (n_row < p.N) {
-        if (p.col_scale) e_sig = p.sigma * ld_nc_f32(p.col_scale + n_row);
-        if (p.bias) e_bias = ld_nc_bf16(p.bias + n_row);
+      {
+        const int n_row = (tile / p.m_tiles) * TILE_N + r;
+        float e_sig = p.sigma, e_bias = 0.f;
+        if (n_row < p.N) {
+          if (p.col_scale) e_sig = p.sigma * ld_nc_f32(p.col_scale + n_row);
+          if (p.bias) e_bias = ld_nc_bf16(p.bias + n_row);
+        }
+        epi[et] = e_sig;
+        epi[256 + et] = e_bias;
       }
       if constexpr (!C::STATIC) {
         // the weight operand needs no x: the first A_STAGES stages are
         // unpacked before the grid-dependency wait has even returned
-        for (int j = 0; j < nst; ++j, ++it) {
-          const int slot = it % C::STAGES;
-          if (!mbar_wait_warp(&full_w[slot], (it / C::STAGES) & 1, ctl())) { ok = false; break; }
-          uint32_t o[32];
-          prologue_stage<FMT, BN>(smem + slot * C::STAGE_BYTES + C::W_OFF, r, h, p.mx_bias, o);
-          const int as = it % C::A_STAGES;
-          if (!mbar_wait_warp(&aempty[as], ((it / C::A_STAGES) & 1) ^ 1, ctl())) { ok = false; break; }
+        for (int j = 0; j < nst; ++j) {
+          if (!mbar_wait_warp(&full_w[ws], wph, ctl())) { ok = false; break; }
+          // unpack the first half while the TMEM slot may still be read by
+          // the MMAs of an earlier stage, then store it, unpack the second
+          // half (after which the weight slot is free) and store it
+          const uint8_t* chunk = w_ring + ws * C::W_SLOT;
+          const uint32_t ta = tmem + lane_base + as * (STAGE_K / 2) + h * 32;
+          uint32_t o[16];
+          prologue_half<FMT>(chunk, r, h, 0, p.mx_bias, o);
+          if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) { ok = false; break; }
           tc_fence_after();
-          tmem_st32(tmem + lane_base + as * (STAGE_K / 2) + h * 32, o);
+          tmem_st16(ta, o);
+          prologue_half<FMT>(chunk, r, h, 1, p.mx_bias, o);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wempty[ws]);
+          tmem_st16(ta + 16, o);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&aready[as]);
+          if (++ws == C::WST) {
+            ws = 0;
+            wph ^= 1;
+          }
+          if (++as == C::A_STAGES) {
+            as = 0;
+            aph ^= 1;
+          }
         }
       } else {
-        for (int j = 0; j < nst; ++j, ++it) {
-          const int slot = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1;
-          if (!mbar_wait_warp(&full_x[slot], ph, ctl())) { ok = false; break; }
-          // the shared e4m3 buffer of this slot is free once its previous MMAs finished
-          if (!mbar_wait_warp(&empty[slot], ph ^ 1, ctl())) { ok = false; break; }
-          uint8_t* st = smem + slot * C::STAGE_BYTES;
-          quantize_x_tile<BN>(st + C::X_OFF, st + C::Q_OFF, p.s_x, threadIdx.x - 64);
+        // static FP8: quantize each x tile into the e4m3 half of its slot
+        // (the slot was refilled only after its previous MMAs completed)
+        for (int j = 0; j < nst; ++j) {
+          if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
+          uint8_t* xd = x_ring + xs * C::X_SLOT;
+          quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, et);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&aready[slot]);
+          if (lane == 0) mbar_arrive(&aready[xs]);
+          if (++xs == C::XST) {
+            xs = 0;
+            xph ^= 1;
+          }
         }
       }
       if (!ok) break;
-
       // ---- epilogue of this tile
       if (!mbar_wait_warp(acc_full, t & 1, ctl())) { ok = false; break; }
       tc_fence_after();
@@ -449,6 +490,8 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // (no grid-dependency wait here: the producer's wait precedes the x
       // loads this accumulator depends on, so every earlier grid is done)
       if (p.split == 1) {
+        const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
+        const float e_sig = epi[et], e_bias = epi[256 + et];
         if (n_row < p.N) {
 #pragma unroll
           for (int i = 0; i < HALF; ++i) {
@@ -463,7 +506,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     if (p.split > 1) {
       // ---- cluster split-K.  Rank q owns the tile's columns
       // [q*BN/S, (q+1)*BN/S).  Each CTA writes its whole partial tile into
-      // its own (now idle) stage buffers as [column][row] fp32, then one
+      // its own (now idle) x ring as [column][row] fp32, then one
       // thread sends every peer the block of that peer's columns with one
       // bulk copy that completes on the peer's red_bar.  The owner adds the
       // S partials of its columns in rank order (deterministic).  Every
@@ -472,7 +515,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       const int q = (int)cluster_rank();
       const int cmax = BN / S;
       const bool good = ok && have_acc;
-      float* part = reinterpret_cast<float*>(smem);   // [BN][TILE_N]; all MMAs are done
+      float* part = reinterpret_cast<float*>(x_ring);   // [BN][TILE_N]; all MMAs are done
       if (good) {
 #pragma unroll
         for (int i = 0; i < HALF; ++i) part[(h * HALF + i) * TILE_N + r] = acc[i];
@@ -491,6 +534,8 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // wait for every peer's partial even after an abort (bounded by the
       // timeout alone)
       const bool ok2 = mbar_wait_warp_cluster(red_bar, 0, ctl_no_abort());
+      const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
+      const float e_sig = epi[et], e_bias = epi[256 + et];
       if (good && ok2 && !*abort_flag && n_row < p.N) {
         const int c0 = q * cmax;
         for (int c = c0 + h; c < c0 + cmax; c += 2) {
@@ -512,7 +557,7 @@ __global__ void __launch_bounds__(352, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     // no CTA leaves while a copy out of or into its shared memory may be in
     // flight: every CTA arrives here only after all its incoming partials
     // landed, so once all have arrived every copy of the cluster is done
-    if (warp < 2 || warp == 10) cluster_wait();   // the epilogue warps waited above
+    if (warp < 2 || warp >= 10) cluster_wait();   // the epilogue warps waited above
     cluster_sync();
   }
   tc_fence_before();
