@@ -69,13 +69,10 @@ struct GemmCfg {
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);    // within an x slot
   static constexpr int W_SLOT = align_up(CHUNK, 1024);
   static constexpr int XST = BN <= 32 ? 3 : 2;
-  // split-K receive buffer: the S - 1 peers' partials of this CTA's BN / S
-  // columns, [peer slot][column][row] fp32 (S divides BN)
-  static constexpr int RECV_BYTES = BN * TILE_N * 4;
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
   static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : 200 * 1024;
-  static constexpr int WST_RAW = (SMEM_BUDGET - XST * X_SLOT - RECV_BYTES - 3072) / W_SLOT;   // barriers, EPI, slack
+  static constexpr int WST_RAW = (SMEM_BUDGET - XST * X_SLOT - 3072) / W_SLOT;   // barriers, EPI, slack
   static constexpr int WST = WST_RAW < 2 ? 2 : (WST_RAW > 8 ? 8 : WST_RAW);
   static constexpr int STAGES = WST;   // weight stages in flight (reported by the plan)
   static constexpr int X_RING_OFF = 0;
@@ -90,8 +87,7 @@ struct GemmCfg {
   static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
   static constexpr int TMEM_COLS = pow2_at_least(A_COLS + ISSUERS * BN);
-  static constexpr int RECV_OFF = W_RING_OFF + WST * W_SLOT;
-  static constexpr int BAR_OFF = RECV_OFF + RECV_BYTES;
+  static constexpr int BAR_OFF = W_RING_OFF + WST * W_SLOT;
   static constexpr int BAR_BYTES = 8 * 40;
   // each epilogue thread's row factor and bias, parked in shared memory over
   // the main loop instead of holding registers: [2][256] fp32
@@ -221,7 +217,6 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* x_ring = smem + C::X_RING_OFF;
   uint8_t* w_ring = smem + C::W_RING_OFF;
-  float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);
   uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [8] weight chunk landed
   uint64_t* wempty = full_w + 8;          // [8] weight slot read (prologue, or MMAs for static FP8)
   uint64_t* full_x = wempty + 8;          // [3] x tile landed
@@ -231,8 +226,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint64_t* acc_full = aempty + 3;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;        // [2], one per MMA issuer
-  uint64_t* red_bar = drain + 2;          // split-K: the peers' partials have landed in recv
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,9 +250,6 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     mbar_init(acc_empty, 8);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
-    mbar_init(red_bar, 1);
-    // the peers' partials arrive as bulk copies counted in bytes
-    if (p.split > 1) mbar_arrive_expect_tx(red_bar, (uint32_t)((p.split - 1) * (BN / p.split) * TILE_N * 4));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -268,9 +259,6 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // split-K: publish this CTA's barriers to the cluster now, wait for the
-  // peers' only right before pushing partials to them
-  if (p.split > 1) cluster_arrive_relaxed();
   pdl_launch_dependents();   // the next call may start its own prologue now
 
   const Work wk = cta_work(p);
@@ -504,12 +492,12 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     if (!ok) *abort_flag = 1;
 
     if (p.split > 1) {
-      // ---- cluster split-K.  Rank q owns the tile's columns
-      // [q*BN/S, (q+1)*BN/S).  Each CTA writes its whole partial tile into
-      // its own (now idle) x ring as [column][row] fp32, then one
-      // thread sends every peer the block of that peer's columns with one
-      // bulk copy that completes on the peer's red_bar.  The owner adds the
-      // S partials of its columns in rank order (deterministic).  Every
+      // ---- cluster split-K.  Every CTA writes its whole partial tile into
+      // its own (now idle) x ring as [column][row] fp32; after one cluster
+      // barrier, rank q reads the tile's columns [q*BN/S, (q+1)*BN/S) of all
+      // S partials (its peers' through distributed shared memory) and adds
+      // them in rank order (deterministic).  A second cluster barrier keeps
+      // every CTA alive until its peers have read its partial.  Every
       // epilogue warp takes part even after an abort.
       const int S = p.split;
       const int q = (int)cluster_rank();
@@ -520,45 +508,35 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
 #pragma unroll
         for (int i = 0; i < HALF; ++i) part[(h * HALF + i) * TILE_N + r] = acc[i];
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 256);
-      cluster_wait();   // the peers' barriers are initialised and armed
-      if (threadIdx.x == 64) {
-        for (int pr = 0; pr < S; ++pr) {
-          if (pr == q) continue;
-          const int slot = q < pr ? q : q - 1;   // this CTA's slot in the peer's recv
-          bulk_s2cluster(dsmem_addr(recv + slot * cmax * TILE_N, pr), part + pr * cmax * TILE_N,
-                         (uint32_t)(cmax * TILE_N * 4), dsmem_addr(red_bar, pr));
-        }
-      }
-      // wait for every peer's partial even after an abort (bounded by the
-      // timeout alone)
-      const bool ok2 = mbar_wait_warp_cluster(red_bar, 0, ctl_no_abort());
+      cluster_sync();   // every partial of the cluster is written (release / acquire)
       const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
       const float e_sig = epi[et], e_bias = epi[256 + et];
-      if (good && ok2 && !*abort_flag && n_row < p.N) {
-        const int c0 = q * cmax;
-        for (int c = c0 + h; c < c0 + cmax; c += 2) {
-          float sum = 0.f;
-          for (int pr = 0; pr < S; ++pr) {
-            const float v = pr == q ? part[c * TILE_N + r]
-                                    : recv[((pr < q ? pr : pr - 1) * cmax + (c - c0)) * TILE_N + r];
-            sum = pr == 0 ? v : sum + v;
-          }
-          const int m = m_tile * BN + c;
-          if (m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
-        }
+      const bool all_good = good && !*abort_flag;
+      const int c0 = q * cmax;
+      for (int c = c0 + h; c < c0 + cmax; c += 2) {
+        // issue the S loads of this output first, then add in rank order
+        float v[8];
+#pragma unroll
+        for (int pr = 0; pr < 8; ++pr)
+          if (pr < S) v[pr] = pr == q ? part[c * TILE_N + r] : ld_dsmem_f32(part + c * TILE_N + r, (uint32_t)pr);
+        float sum = v[0];
+#pragma unroll
+        for (int pr = 1; pr < 8; ++pr)
+          if (pr < S) sum += v[pr];
+        const int m = m_tile * BN + c;
+        if (all_good && n_row < p.N && m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
       }
     }
   }
 
   __syncwarp();
   if (p.split > 1) {
-    // no CTA leaves while a copy out of or into its shared memory may be in
-    // flight: every CTA arrives here only after all its incoming partials
-    // landed, so once all have arrived every copy of the cluster is done
-    if (warp < 2 || warp >= 10) cluster_wait();   // the epilogue warps waited above
-    cluster_sync();
+    // the non-epilogue warps take the first cluster barrier here; then no CTA
+    // leaves before its peers have read its partial (their reads completed
+    // before they arrive, so the arrive needs no release)
+    if (warp < 2 || warp >= 10) cluster_sync();
+    cluster_arrive_relaxed();
+    cluster_wait();
   }
   tc_fence_before();
   __syncthreads();
