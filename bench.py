@@ -488,6 +488,30 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 
 
+def run_ncu_case(fmt):
+    """Eight back-to-back calls of one format at the step's Linear shape,
+    rotating over four weight sets: the case the committed ncu captures take
+    (one launch, after four warm ones)."""
+    import torch
+
+    import weight_only_quantized_prologue_b200 as dq
+    from weight_only_quantized_prologue_b200 import synthetic
+
+    torch.cuda.set_device(0)
+    layers = []
+    for r in range(4):
+        x, w, b = synthetic.linear_inputs(LM, LK, LN, seed=r)
+        layers.append(dq.QuantizedLinear.from_float(fmt, w.cuda(), b.cuda()))
+    xc = x.cuda()
+    y = torch.empty((LM, LN), dtype=torch.bfloat16, device="cuda")
+    for i in range(8):
+        layers[i % 4](xc, out=y)
+    torch.cuda.synchronize()
+    for l in layers:
+        assert l.last_error() == 0, "device-side wait timed out"
+    print(json.dumps({"ncu_case": fmt, "M": LM, "K": LK, "N": LN, "plan": layers[0].plan(LM)}), flush=True)
+
+
 def run_sweep(args):
     import torch
 
@@ -561,6 +585,9 @@ def main():
     ap.add_argument("--sweep-m", default="1,16,32,128,1024,4096")
     ap.add_argument("--sweep-kn", default="4096x4096,4096x14336,14336x4096")
     ap.add_argument("--sweep-formats", default="int4,nvfp4,mxfp4,fp8,fp8_static")
+    ap.add_argument("--ncu-case", choices=list(LIN_FORMATS), default=None,
+                    help="small profiling case: 8 plain launches of one format at the step's shape "
+                         "(4 weight sets, no graphs, no timing) for an ncu capture")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -570,6 +597,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.ncu_case:
+        run_ncu_case(args.ncu_case)
         return
 
     if args.impl == "reference":

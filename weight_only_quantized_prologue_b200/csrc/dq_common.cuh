@@ -117,34 +117,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, c
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
-      : "memory");
-  return ok != 0;
-}
 
-// Whole-warp wait for data other CTAs of the cluster pushed into this CTA
-// (acquire at cluster scope); bounded like mbar_wait.
-__device__ __forceinline__ bool mbar_wait_cluster_slow(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (wait_give_up(ctl, t0)) return false;
-  }
-}
-__device__ __forceinline__ bool mbar_wait_warp_cluster(uint64_t* bar, uint32_t parity, const WaitCtl ctl) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster_slow(bar, parity, ctl) ? 1 : 0;
-  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-  if (ok) mbar_try_wait_cluster(bar, parity);
-  return ok != 0;
-}
 
 // ---------------------------------------------------------------------------
 // bulk and tensor copies global -> shared (no multicast anywhere)
@@ -213,20 +186,6 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-// shared::cluster address of `local` in the CTA of rank `rank`
-__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  return remote;
-}
-__device__ __forceinline__ void st_dsmem_f32(uint32_t remote, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
-}
-// arrive on an mbarrier of another CTA of the cluster, releasing this
-// thread's prior (distributed) shared-memory writes at cluster scope
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
 __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
@@ -234,25 +193,7 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
   return v;
 }
-__device__ __forceinline__ float4 ld_dsmem_f32x4(const void* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(remote)
-               : "memory");
-  return v;
-}
 
-// Bulk copy from this CTA's shared memory into another CTA of the cluster;
-// completes `bytes` of transaction count on the destination's mbarrier
-// (both given as shared::cluster addresses).  No multicast.
-__device__ __forceinline__ void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "r"(smem_u32(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
 // named barrier over a subset of the CTA's warps
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

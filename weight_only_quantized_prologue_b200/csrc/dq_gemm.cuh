@@ -512,19 +512,28 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
       const float e_sig = epi[et], e_bias = epi[256 + et];
       const bool all_good = good && !*abort_flag;
+      // This thread's HALF values are the S partials of columns
+      // c0 + h + 2 * ci, ci < cmax / 2 (S * cmax / 2 = HALF): all the loads
+      // are issued first, then each column is added in rank order.
       const int c0 = q * cmax;
-      for (int c = c0 + h; c < c0 + cmax; c += 2) {
-        // issue the S loads of this output first, then add in rank order
-        float v[8];
+      const int lg_s = __ffs(S) - 1;   // S is a power of two
+      float v[HALF];
 #pragma unroll
-        for (int pr = 0; pr < 8; ++pr)
-          if (pr < S) v[pr] = pr == q ? part[c * TILE_N + r] : ld_dsmem_f32(part + c * TILE_N + r, (uint32_t)pr);
-        float sum = v[0];
+      for (int i = 0; i < HALF; ++i) {
+        const int pr = i & (S - 1);
+        const int c = c0 + h + 2 * (i >> lg_s);
+        v[i] = pr == q ? part[c * TILE_N + r] : ld_dsmem_f32(part + c * TILE_N + r, (uint32_t)pr);
+      }
+      float sum = 0.f;
 #pragma unroll
-        for (int pr = 1; pr < 8; ++pr)
-          if (pr < S) sum += v[pr];
-        const int m = m_tile * BN + c;
-        if (all_good && n_row < p.N && m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
+      for (int i = 0; i < HALF; ++i) {
+        const int pr = i & (S - 1);
+        sum = pr == 0 ? v[i] : sum + v[i];
+        if (pr == S - 1) {
+          const int m = m_tile * BN + c0 + h + 2 * (i >> lg_s);
+          if (all_good && n_row < p.N && m < p.M)
+            p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
+        }
       }
     }
   }
