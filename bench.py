@@ -306,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
         for l in list(s.layers.values()) + [s.mlp1, s.mlp2]:
             assert l.last_error() == 0, "device-side wait timed out"
 
-    value = ms * 1000.0 / (args.steps * CALLS_PER_STEP * world)
+    value = job_us_per_call(ms, args.steps, CALLS_PER_STEP, world)
     peaks = measured_peaks()
     lin = {n: per_call[n] for n in LIN_FORMATS}
     dom = max(lin, key=lin.get)
@@ -333,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}", "timing": "CUDA graphs, CUDA events"},
         "per_call": per_format,
         "roofline": roofline,
-        "e2e": {"value": round(e2e_ms * 1000.0 / (e2e_steps * CALLS_PER_STEP * world), 4), "unit": UNIT,
+        "e2e": {"value": round(job_us_per_call(e2e_ms, e2e_steps, CALLS_PER_STEP, world), 4), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps * CALLS_PER_STEP,
         "clocks": clocks,
@@ -350,6 +350,12 @@ def _e2e_step(s, host):
         layer(x, out=y)
         if name in hy:
             hy[name].copy_(y, non_blocking=True)
+
+
+def job_us_per_call(ms_max, steps, calls_per_step, world):
+    """Whole-job time per call: every rank runs `steps` steps of
+    `calls_per_step` calls; the job takes the slowest rank's time."""
+    return ms_max * 1000.0 / (steps * calls_per_step * world)
 
 
 def aggregate_max(v):
