@@ -100,6 +100,16 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt, int K, int N,
  * synchronized. */
 dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream);
 
+/* DQ_FP8_STATIC only: the GEMM on activations already quantized by
+ * dqgemm_quantize_act_fp8 with the handle's s_x (the static page's "Graph
+ * after export": the Q node's e4m3 output feeds the FP8 GEMM).  q: device u8
+ * [M, K] e4m3 codes, row-major, 16-byte aligned; y as in dqgemm_run.  The
+ * result is bit-identical to dqgemm_run on the x that q was quantized from;
+ * the in-kernel quantization of dqgemm_run is repeated for every 128-channel
+ * tile, so for larger M (about 128 rows and up) quantizing once and calling
+ * this is faster.  DQ_ERR_UNSUPPORTED for other formats. */
+dqgemm_status dqgemm_run_fp8_static_quantized(dqgemm_handle h, const void* q, int M, void* y, void* stream);
+
 /* Release the handle and its device memory (synchronizes the device). */
 dqgemm_status dqgemm_destroy(dqgemm_handle h);
 

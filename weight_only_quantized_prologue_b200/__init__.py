@@ -24,6 +24,7 @@ from ._native import (  # noqa: F401
     dqgemm_pack_host,
     dqgemm_quantize_act_fp8,
     dqgemm_run,
+    dqgemm_run_fp8_static_quantized,
     dqgemm_selftest_timeout,
     dqgemm_status_string,
     storage_shapes,
@@ -37,8 +38,13 @@ class QuantizedLinear:
     ``fmt`` (see ``storage_shapes``); they are copied and re-laid-out by the
     library, so the caller may drop them afterwards."""
 
+    # static FP8 from this many rows on: quantize x once, then the FP8 GEMM
+    # (the fused kernel re-quantizes x for every 128-channel tile)
+    STATIC_PREQUANT_M = 128
+
     def __init__(self, fmt, K, N, packed, scales, global_scale=1.0, bias=None):
         self.fmt, self.K, self.N = fmt, K, N
+        self.act_scale = float(global_scale) if fmt == "fp8_static" else None
         self._h = dqgemm_create(fmt, K, N, packed, scales, global_scale, bias)
 
     @classmethod
@@ -63,7 +69,12 @@ class QuantizedLinear:
         M = x.shape[0]
         if out is None:
             out = torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
-        dqgemm_run(self._h, x, M, out, stream)
+        if self.fmt == "fp8_static" and M >= self.STATIC_PREQUANT_M:
+            q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
+            dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
+            dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)
+        else:
+            dqgemm_run(self._h, x, M, out, stream)
         return out
 
     def dequantize(self, stream=None):

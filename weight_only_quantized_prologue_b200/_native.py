@@ -41,6 +41,7 @@ _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _SIGNATURES = {
     "dqgemm_create": [ctypes.POINTER(_VP), _I, _I, _I, _VP, _VP, _F, _VP],
     "dqgemm_run": [_VP, _VP, _I, _VP, _VP],
+    "dqgemm_run_fp8_static_quantized": [_VP, _VP, _I, _VP, _VP],
     "dqgemm_destroy": [_VP],
     "dqgemm_dequantize": [_VP, _VP, _VP],
     "dqgemm_quantize_act_fp8": [_VP, _I, _I, _F, _VP, _VP],
@@ -118,6 +119,11 @@ def dqgemm_create(fmt, K, N, packed_w, scales, global_scale=1.0, bias=None):
 
 def dqgemm_run(h, x, M, y, stream=None):
     _check(lib().dqgemm_run(h, _ptr(x), int(M), _ptr(y), _stream(stream)), "dqgemm_run")
+
+
+def dqgemm_run_fp8_static_quantized(h, q, M, y, stream=None):
+    _check(lib().dqgemm_run_fp8_static_quantized(h, _ptr(q), int(M), _ptr(y), _stream(stream)),
+           "dqgemm_run_fp8_static_quantized")
 
 
 def dqgemm_destroy(h):

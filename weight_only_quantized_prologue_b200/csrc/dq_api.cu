@@ -199,6 +199,20 @@ bool make_x_map(CUtensorMap* map, const void* x, int M, int K, int bn, bool* is3
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// e4m3 activations [M, K] (u8, K % 16 == 0): box of 128 k x bn rows, the
+// tensor core's 128-byte-swizzled K-major image
+bool make_q_map(CUtensorMap* map, const void* q, int M, int K, int bn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)K};
+  const cuuint32_t box[2] = {128, (cuuint32_t)bn};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // launch dispatch
 // ---------------------------------------------------------------------------
@@ -483,14 +497,14 @@ dqgemm_status dqgemm_get_plan(dqgemm_handle h, int M, dqgemm_plan* plan) {
   return DQ_OK;
 }
 
-dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream) {
+static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, void* y, void* stream) {
   if (!h || !x || !y || M < 1) return DQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
   dqgemm_plan pl;
   fill_plan(h, M, &pl);
   CUtensorMap tm;
   bool x3d = false;
-  if (!make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
+  if (xq ? !make_q_map(&tm, x, M, h->K, pl.bn) : !make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
   GemmParams p;
   p.wchunks = h->wchunks;
   p.col_scale = h->col_scale;
@@ -507,11 +521,22 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
   p.tiles = pl.m_tiles * pl.n_tiles;
   p.split = pl.max_segments;
   p.x3d = x3d ? 1 : 0;
+  p.xq = xq ? 1 : 0;
   p.timeout_ns = timeout_ns();
   cudaError_t e = cudaSuccess;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   DQ_FMT_SWITCH(h->fmt, e = launch_fmt<F>(pl.bn, tm, p, pl.grid, s));
   return cuda_err(e);
+}
+
+dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream) {
+  return run_gemm(h, x, false, M, y, stream);
+}
+
+dqgemm_status dqgemm_run_fp8_static_quantized(dqgemm_handle h, const void* q, int M, void* y, void* stream) {
+  if (!h) return DQ_ERR_INVALID_ARG;
+  if (h->fmt != FMT_FP8S) return DQ_ERR_UNSUPPORTED;
+  return run_gemm(h, q, true, M, y, stream);
 }
 
 dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream) {

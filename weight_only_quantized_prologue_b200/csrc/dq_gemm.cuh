@@ -47,6 +47,8 @@ struct GemmParams {
   int tiles;                     // n_tiles * m_tiles
   int split;                     // CTAs per tile (cluster size); 1 = whole tiles
   int x3d;                       // x map is 3-D {64, M, K/64}: one box per stage
+  int xq;                        // static FP8: x arrives already quantized, e4m3 [M, K]
+                                 // through a 2-D u8 map (box 128 k x BN rows)
   unsigned long long timeout_ns;
 };
 
@@ -308,12 +310,18 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         for (int ks = wk.kb; ks < wk.ke; ++ks, ++it) {
           if (it >= C::XST && !mbar_wait(&xempty[xs], xph ^ 1, ctl())) { ok = false; break; }
           uint8_t* xd = x_ring + xs * C::X_SLOT;
-          mbar_arrive_expect_tx(&full_x[xs], C::X_BYTES);
-          if (p.x3d) {
-            tma_load_3d(xd, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[xs]);
+          if (C::STATIC && p.xq) {
+            // e4m3 codes straight into the operand half of the slot
+            mbar_arrive_expect_tx(&full_x[xs], C::Q_BYTES);
+            tma_load_2d(xd + C::Q_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
           } else {
-            tma_load_2d(xd, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
-            tma_load_2d(xd + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[xs]);
+            mbar_arrive_expect_tx(&full_x[xs], C::X_BYTES);
+            if (p.x3d) {
+              tma_load_3d(xd, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[xs]);
+            } else {
+              tma_load_2d(xd, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
+              tma_load_2d(xd + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[xs]);
+            }
           }
           if (++xs == C::XST) {
             xs = 0;
@@ -444,12 +452,15 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         }
       } else {
         // static FP8: quantize each x tile into the e4m3 half of its slot
-        // (the slot was refilled only after its previous MMAs completed)
+        // (the slot was refilled only after its previous MMAs completed);
+        // pre-quantized x is only passed on
         for (int j = 0; j < nst; ++j) {
           if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
-          uint8_t* xd = x_ring + xs * C::X_SLOT;
-          quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, et);
-          fence_proxy_async_smem();
+          if (!p.xq) {
+            uint8_t* xd = x_ring + xs * C::X_SLOT;
+            quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, et);
+            fence_proxy_async_smem();
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&aready[xs]);
           if (++xs == C::XST) {
