@@ -485,6 +485,7 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   if (e == cudaSuccess && h->col_scale) e = cudaMemcpy(h->col_scale, hs.data(), (size_t)N * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && h->bias) e = cudaMemcpy(h->bias, bias, (size_t)N * 2, cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) { DQ_FMT_SWITCH(fmt, e = set_attrs<F>()); }
+  if (e == cudaSuccess && fmt == FMT_FP8S) e = set_attrs<FMT_FP8SQ>();
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) { dqgemm_destroy(h); return DQ_ERR_CUDA; }
   *out = h;
@@ -521,11 +522,14 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   p.tiles = pl.m_tiles * pl.n_tiles;
   p.split = pl.max_segments;
   p.x3d = x3d ? 1 : 0;
-  p.xq = xq ? 1 : 0;
   p.timeout_ns = timeout_ns();
   cudaError_t e = cudaSuccess;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  DQ_FMT_SWITCH(h->fmt, e = launch_fmt<F>(pl.bn, tm, p, pl.grid, s));
+  if (xq) {
+    e = launch_fmt<FMT_FP8SQ>(pl.bn, tm, p, pl.grid, s);
+  } else {
+    DQ_FMT_SWITCH(h->fmt, e = launch_fmt<F>(pl.bn, tm, p, pl.grid, s));
+  }
   return cuda_err(e);
 }
 

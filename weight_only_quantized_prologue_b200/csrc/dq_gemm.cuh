@@ -47,8 +47,6 @@ struct GemmParams {
   int tiles;                     // n_tiles * m_tiles
   int split;                     // CTAs per tile (cluster size); 1 = whole tiles
   int x3d;                       // x map is 3-D {64, M, K/64}: one box per stage
-  int xq;                        // static FP8: x arrives already quantized, e4m3 [M, K]
-                                 // through a 2-D u8 map (box 128 k x BN rows)
   unsigned long long timeout_ns;
 };
 
@@ -59,9 +57,12 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 
 template <int FMT, int BN>
 struct GemmCfg {
-  static constexpr bool STATIC = (FMT == FMT_FP8S);
+  // static FP8 with x quantized beforehand: x arrives as e4m3 [M, K] through
+  // a 2-D u8 map (box 128 k x BN rows), straight into the operand buffer
+  static constexpr bool XQ = (FMT == FMT_FP8SQ);
+  static constexpr bool STATIC = (FMT == FMT_FP8S) || XQ;
   static constexpr int CHUNK = chunk_bytes(FMT);
-  static constexpr int X_BYTES = BN * 256;                 // two 64-k blocks of BN rows x 128 B
+  static constexpr int X_BYTES = XQ ? 0 : BN * 256;        // two 64-k blocks of BN rows x 128 B
   static constexpr int Q_BYTES = STATIC ? BN * 128 : 0;    // e4m3 x tile (static FP8)
   // Two rings: packed weight chunks (streamed from the start of the kernel;
   // a slot is free once the prologue has read it, or for static FP8 once the
@@ -103,7 +104,7 @@ struct GemmCfg {
   static_assert(A_COLS + ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");   // (two CTAs per SM need <= 113 KB)
   static_assert(A_STAGES <= 3 && XST <= 3, "barrier arrays");
-  static_assert(XST * X_SLOT >= BN * TILE_N * 4, "split-K partial tile fits in the x ring");
+  static_assert(XST * X_SLOT + WST * W_SLOT >= BN * TILE_N * 4, "split-K partial tile fits in the rings");
 };
 
 // The work of one CTA: a list of (tile, k_begin, k_end) segments.
@@ -310,8 +311,8 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         for (int ks = wk.kb; ks < wk.ke; ++ks, ++it) {
           if (it >= C::XST && !mbar_wait(&xempty[xs], xph ^ 1, ctl())) { ok = false; break; }
           uint8_t* xd = x_ring + xs * C::X_SLOT;
-          if (C::STATIC && p.xq) {
-            // e4m3 codes straight into the operand half of the slot
+          if constexpr (C::XQ) {
+            // e4m3 codes straight into the operand buffer of the slot
             mbar_arrive_expect_tx(&full_x[xs], C::Q_BYTES);
             tma_load_2d(xd + C::Q_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
           } else {
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         // pre-quantized x is only passed on
         for (int j = 0; j < nst; ++j) {
           if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
-          if (!p.xq) {
+          if constexpr (!C::XQ) {
             uint8_t* xd = x_ring + xs * C::X_SLOT;
             quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, et);
             fence_proxy_async_smem();
@@ -504,7 +505,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
 
     if (p.split > 1) {
       // ---- cluster split-K.  Every CTA writes its whole partial tile into
-      // its own (now idle) x ring as [column][row] fp32; after one cluster
+      // its own (now idle) rings as [column][row] fp32; after one cluster
       // barrier, rank q reads the tile's columns [q*BN/S, (q+1)*BN/S) of all
       // S partials (its peers' through distributed shared memory) and adds
       // them in rank order (deterministic).  A second cluster barrier keeps
@@ -514,7 +515,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       const int q = (int)cluster_rank();
       const int cmax = BN / S;
       const bool good = ok && have_acc;
-      float* part = reinterpret_cast<float*>(x_ring);   // [BN][TILE_N]; all MMAs are done
+      float* part = reinterpret_cast<float*>(smem);   // [BN][TILE_N] over both rings; all MMAs are done
       if (good) {
 #pragma unroll
         for (int i = 0; i < HALF; ++i) part[(h * HALF + i) * TILE_N + r] = acc[i];

@@ -39,7 +39,10 @@
 
 namespace dq {
 
-enum Fmt { FMT_INT4 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_FP8S = 4 };
+enum Fmt { FMT_INT4 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_FP8S = 4,
+           // static FP8 GEMM fed with activations quantized beforehand (same
+           // weight chunks as FMT_FP8S; a kernel variant, not a storage format)
+           FMT_FP8SQ = 5 };
 
 constexpr int TILE_N = 128;      // output channels per tile (MMA M)
 constexpr int STAGE_K = 128;     // k per pipeline stage (= one INT4 group)
