@@ -1,7 +1,8 @@
 """Host-side checks of the C ABI (no GPU needed): the library loads and
 exports every entry point include/dqgemm.h declares, the host packer is
 bit-identical to the oracle, argument errors come back as status codes, and
-the stream-K partition arithmetic covers every unit exactly once."""
+the split-K arithmetic of the GEMM (K-stage ranges per rank, the owner's
+reads of the partial tiles) covers everything exactly once, in rank order."""
 
 import ctypes
 import os
@@ -97,26 +98,48 @@ def test_entry_points_reject_null_arguments_without_touching_the_gpu():
     assert dq.dqgemm_status_string(6) == "DQ_ERR_TIMEOUT"
 
 
-# -- stream-K partition: the arithmetic the kernel and the planner share ----
+# -- split-K: the arithmetic of dq_gemm_kernel's cluster split -------------
 
 
-def _cta_of_unit(u, U, G):
-    return ((u + 1) * G - 1) // U
+def _stage_range(q, KS, S):
+    """K stages of rank q (cta_work): [q*KS/S, (q+1)*KS/S)."""
+    return q * KS // S, (q + 1) * KS // S
 
 
-def _cta_start(c, U, G):
-    return c * U // G
+@pytest.mark.parametrize("S", [2, 4, 8])
+@pytest.mark.parametrize("KS", [2, 3, 8, 24, 25, 112])
+def test_split_k_stage_ranges_cover_k_once(S, KS):
+    if S > KS:                 # the planner never splits deeper than k_stages
+        return
+    seen = np.zeros(KS, dtype=int)
+    for q in range(S):
+        a, b = _stage_range(q, KS, S)
+        assert b > a
+        seen[a:b] += 1
+    assert (seen == 1).all()
 
 
-@pytest.mark.parametrize("U,G", [(768, 148), (148, 148), (149, 148), (32768, 148), (7, 7), (5000, 37), (24, 148)])
-def test_stream_k_partition_covers_every_unit_once(U, G):
-    G = min(G, U)
-    owner = np.full(U, -1)
-    for c in range(G):
-        a, b = _cta_start(c, U, G), _cta_start(c + 1, U, G)
-        assert b > a                       # no empty range when G <= U
-        assert (owner[a:b] == -1).all()
-        owner[a:b] = c
-    assert (owner >= 0).all()
-    for u in range(U):
-        assert _cta_of_unit(u, U, G) == owner[u]
+def _owner_reads(q, h, BN, S):
+    """(rank, column) pairs that thread half h of rank q reads, in the order
+    it adds them: value i is rank i % S of column c0 + h + 2 * (i // S)."""
+    cmax, c0 = BN // S, q * (BN // S)
+    return [(i % S, c0 + h + 2 * (i // S)) for i in range(BN // 2)]
+
+
+@pytest.mark.parametrize("BN", [16, 32, 64, 128])
+@pytest.mark.parametrize("S", [2, 4, 8])
+def test_split_k_owners_read_every_partial_once_in_rank_order(BN, S):
+    got = {}
+    for q in range(S):
+        owned = set(range(q * BN // S, (q + 1) * BN // S))
+        for h in range(2):
+            reads = _owner_reads(q, h, BN, S)
+            for k, (pr, c) in enumerate(reads):
+                assert c in owned                      # only its own columns
+                assert (pr, c) not in got              # each partial value once
+                got[(pr, c)] = (q, h, k)
+            # each column's S values are consecutive and in rank order 0..S-1
+            for j in range(0, len(reads), S):
+                assert [pr for pr, _ in reads[j:j + S]] == list(range(S))
+                assert len({c for _, c in reads[j:j + S]}) == 1
+    assert len(got) == S * BN                          # every rank x column
