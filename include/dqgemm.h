@@ -186,7 +186,7 @@ typedef struct {
   int max_segments;     /* most CTAs sharing one output tile (split-K depth) */
   int stages;           /* shared-memory pipeline depth */
   int smem_bytes;       /* dynamic shared memory per CTA */
-  long long workspace_bytes; /* split-K partial buffer the plan needs */
+  long long workspace_bytes; /* global split-K scratch the plan needs (0: partials stay on chip) */
   long long weight_bytes;    /* packed weight + scale bytes streamed per call */
 } dqgemm_plan;
 

@@ -5,13 +5,16 @@
 // rows are its N (BN = 16..128): the skinny decode shapes the quantized-Linear
 // pages run (x of 32 rows) keep the tensor core busy on the weight side.
 //
-// CTA = 11 warps, warp-specialized:
-//   warp 0      producer: one 1-D bulk copy of the stage's pre-tiled weight
-//               chunk + the TMA box load(s) of the bf16 x tile, per stage
+// CTA = 12 warps, warp-specialized:
+//   warp 0      weight producer: one 1-D bulk copy of the stage's pre-tiled
+//               weight chunk per stage into a ring of up to 8 slots, from
+//               CTA entry on (weights never depend on the previous grid)
+//   warp 11     x producer: after the grid-dependency wait, the TMA box
+//               load(s) of the stage's x tile into a 2-3 slot ring
 //   warps 1, 10 MMA issuers: one thread each issues tcgen05.mma for half of
 //               every stage's k-steps into its own TMEM accumulator (a single
 //               thread issues only one MMA every ~80 cycles) and commits the
-//               stage / operand / accumulator barriers
+//               slot / operand / accumulator barriers
 //   warps 2..9  the prologue: unpack + scale the packed codes of one weight
 //               row per thread (two threads per row, one per k-half) into
 //               bf16 operands written straight to TMEM (the MMA reads A from
@@ -20,9 +23,11 @@
 //               accumulators, scale, bias, bf16 cast, store).
 // Work split: a tile of 128 output channels x BN activation rows is either
 // computed whole by one CTA (persistent loop over tiles), or its K range is
-// split over the S CTAs of a thread-block cluster whose fp32 partials are
-// summed through distributed shared memory in rank order (deterministic, no
-// global scratch).
+// split over the S CTAs of a thread-block cluster: each writes its fp32
+// partial tile into its own shared memory and, after a cluster barrier, rank
+// q reads its share of the columns from all S partials over distributed
+// shared memory and adds them in rank order (deterministic, no global
+// scratch).
 // Back-to-back calls overlap through programmatic dependent launch: a CTA
 // sets up and starts streaming its (read-only) weights before waiting for the
 // previous grid; it reads x and writes y only after that wait.
