@@ -1,0 +1,60 @@
+"""nn.Linear drop-in: quantize_ on a bf16 model gives exactly what the
+library's layers give on the same inputs (bit-identical), any leading dims."""
+
+import pytest
+import torch
+
+import weight_only_quantized_prologue_b200 as dq
+from weight_only_quantized_prologue_b200 import module as M
+from weight_only_quantized_prologue_b200 import synthetic
+
+pytestmark = pytest.mark.gpu
+
+
+def _model(seed):
+    torch.manual_seed(seed)
+    m = torch.nn.Sequential(torch.nn.Linear(256, 512), torch.nn.ReLU(), torch.nn.Linear(512, 128))
+    return m.to(device="cuda", dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4", "fp8"])
+def test_quantize_matches_library_layers(fmt):
+    model = _model(1)
+    w1, b1 = model[0].weight.float(), model[0].bias
+    w2, b2 = model[2].weight.float(), model[2].bias
+    l1 = dq.QuantizedLinear.from_float(fmt, w1, b1)
+    l2 = dq.QuantizedLinear.from_float(fmt, w2, b2)
+    M.quantize_(model, fmt)
+    assert isinstance(model[0], M.DQLinear) and isinstance(model[2], M.DQLinear)
+    x = synthetic.activations(2 * 24, 256, seed=5).cuda().view(2, 24, 256)   # leading dims
+    with torch.no_grad():
+        y = model(x)
+    ref = l2(torch.relu(l1(x.view(-1, 256)))).view(2, 24, 128)
+    torch.cuda.synchronize()
+    assert y.shape == (2, 24, 128)
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    l1.close()
+    l2.close()
+
+
+def test_static_fp8_calibrate_then_quantize():
+    model = _model(2)
+    batches = [synthetic.activations(32, 256, seed=s).cuda() for s in range(1, 11)]
+    scales = M.calibrate_static_fp8(model, batches)
+    w1, w2 = model[0].weight.float(), model[2].weight.float()
+    l1 = dq.QuantizedLinear.from_float("fp8_static", w1, model[0].bias, act_scale=scales["0"])
+    l2 = dq.QuantizedLinear.from_float("fp8_static", w2, model[2].bias, act_scale=scales["2"])
+    M.quantize_(model, "fp8_static", act_scales=scales)
+    x = synthetic.activations(160, 256, seed=11).cuda()      # >= 128 rows: quantize-once path
+    with torch.no_grad():
+        y = model(x)
+    ref = l2(torch.relu(l1(x)))
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+    l1.close()
+    l2.close()
+
+
+def test_static_fp8_without_scales_is_refused():
+    with pytest.raises(ValueError):
+        M.quantize_(_model(3), "fp8_static")
