@@ -31,23 +31,43 @@ from .quant import (
     pack_nibbles,
     quantize_fp8_rows,
     quantize_int4,
+    quantize_int4_asym,
     quantize_mxfp4,
     quantize_nvfp4,
     unpack_nibbles,
 )
 
-FORMATS = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static")
+FORMATS = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static", "int4_asym")
+
+
+def asym_scales_pack(scale_bits, zeros):
+    """The canonical scale storage of asymmetric INT4: the bf16 scales
+    [N, G] (little-endian bytes, row-major) followed by the zero points
+    [N, G], as one uint8 array of 3 * N * G bytes."""
+    s = np.ascontiguousarray(scale_bits, dtype="<u2").view(np.uint8).reshape(-1)
+    return np.concatenate([s, np.ascontiguousarray(zeros, dtype=np.uint8).reshape(-1)])
+
+
+def asym_scales_split(buf, N, G):
+    """Inverse of asym_scales_pack: (scale bits uint16 [N, G], zeros uint8 [N, G])."""
+    buf = np.ascontiguousarray(buf, dtype=np.uint8).reshape(-1)
+    s = buf[: 2 * N * G].view("<u2").reshape(N, G)
+    return s, buf[2 * N * G: 3 * N * G].reshape(N, G)
 
 
 def quantize_pack(fmt, W):
     """Quantize W [N, K] and return the storage arrays of the library's
     canonical layout as a dict: ``packed`` (uint8 [N, K/2] for 4-bit formats,
     [N, K] for FP8), ``scales`` (INT4: uint16 bf16 bits [N, K/128]; NVFP4:
-    uint8 E4M3 [N, K/16]; MXFP4: uint8 E8M0 [N, K/32]; FP8: float32 [N]) and
-    ``global_scale`` (NVFP4's g, else 1.0)."""
+    uint8 E4M3 [N, K/16]; MXFP4: uint8 E8M0 [N, K/32]; FP8: float32 [N];
+    asymmetric INT4: asym_scales_pack of the bf16 scales and the zero points)
+    and ``global_scale`` (NVFP4's g, else 1.0)."""
     if fmt == "int4":
         codes, s = quantize_int4(W)
         return dict(packed=pack_nibbles(codes), scales=s, global_scale=1.0)
+    if fmt == "int4_asym":
+        codes, s, z = quantize_int4_asym(W)
+        return dict(packed=pack_nibbles(codes), scales=asym_scales_pack(s, z), global_scale=1.0)
     if fmt == "nvfp4":
         codes, sb, g = quantize_nvfp4(W)
         return dict(packed=pack_nibbles(codes), scales=sb, global_scale=g)
@@ -69,6 +89,12 @@ def dequant_exact(fmt, packed, scales, global_scale=1.0):
         c = unpack_nibbles(packed, signed=True).astype(np.float64)
         s = np.repeat(bf16_from_bits(scales), INT4_GROUP, axis=1)
         return c * s
+    if fmt == "int4_asym":
+        u = unpack_nibbles(packed).astype(np.float64)
+        N = u.shape[0]
+        sb, z = asym_scales_split(scales, N, u.shape[1] // INT4_GROUP)
+        s = np.repeat(bf16_from_bits(sb), INT4_GROUP, axis=1)
+        return (u - np.repeat(z.astype(np.float64), INT4_GROUP, axis=1)) * s
     if fmt == "nvfp4":
         v = e2m1_decode(unpack_nibbles(packed))
         sb = np.repeat(e4m3_decode(scales), NVFP4_BLOCK, axis=1)
@@ -85,12 +111,13 @@ def dequant_exact(fmt, packed, scales, global_scale=1.0):
 def dequant_bf16_bits(fmt, packed, scales, global_scale=1.0):
     """The debug dequantization to bf16, as uint16 bit patterns [N, K]:
       INT4   bf16(c * s)                    (c * s is exact in fp32)
+      INT4 asymmetric  bf16((c - z) * s)    (exact in fp32 as well)
       NVFP4  bf16(f32(e2m1 * dec(sb) * g))  (e2m1 * dec(sb) is exact)
       MXFP4  bf16(e2m1 * 2**(e-127))
       FP8    bf16(f32(e4m3 * s[n]))
     -0.0 is kept (a negative code times a positive scale, or code -0).
     Parity: pinned by brute force over code x scale pairs in the tests."""
-    if fmt == "int4":
+    if fmt in ("int4", "int4_asym"):
         return bf16_bits(bf16(dequant_exact(fmt, packed, scales)))
     if fmt == "nvfp4":
         v = e2m1_decode(unpack_nibbles(packed))

@@ -70,6 +70,41 @@ def quantize_int4(W, group=INT4_GROUP):
     return q.astype(np.int8), bf16_bits(s)
 
 
+def quantize_int4_asym(W, group=INT4_GROUP):
+    """Asymmetric group-wise INT4 with a per-group zero point: the
+    zero-point counterpart of "TorchAO INT4 Weight-Only Quantization
+    (Linear)" (that page's quantizer is the symmetric one, zero-point 0).
+
+    Per row n and group j of ``group`` consecutive k:
+      lo = min(0, min W),  hi = max(0, max W);  s = bf16(f32((hi - lo) / 15));
+      z = clamp(RNE(f32(-lo / s)), 0, 15);
+      code = clamp(RNE(f32(W / s)) + z, 0, 15)  (unsigned);
+      dequantized weight (code - z) * s;  a group with s == 0 has codes 0, z 0.
+    Readings (no page gives them): the range includes 0 so that zero is
+    exactly representable, the scale is bf16 like the symmetric format's,
+    the zero point an integer in [0, 15].
+
+    Returns (codes uint8 [N, K], scale bits uint16 [N, K/group], zero points
+    uint8 [N, K/group]).
+    Parity: pinned by the on-grid round trip (weights built as
+    (c - z) * s with every c in 0..15 quantize back to exactly c, z, s), by
+    the all-zero and non-negative special cases, and by idempotence.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    B = _blocks(W, group)
+    lo = np.minimum(B.min(axis=2), 0.0)
+    hi = np.maximum(B.max(axis=2), 0.0)
+    s = bf16(f32((hi - lo) / 15.0))
+    safe = np.where(s > 0, s, 1.0)
+    z = np.clip(np.rint(f32(-lo / safe)), 0, 15)
+    z = np.where(s > 0, z, 0.0)
+    s_full = np.repeat(safe, group, axis=1)
+    z_full = np.repeat(z, group, axis=1)
+    q = np.clip(np.rint(f32(W / s_full)) + z_full, 0, 15)
+    q = np.where(np.repeat(s, group, axis=1) > 0, q, 0.0)
+    return q.astype(np.uint8), bf16_bits(s), z.astype(np.uint8)
+
+
 def quantize_nvfp4(W):
     """NVFP4 ("TorchAO NVFP4 Weight-Only Quantization (Linear)", intro:
     packed FP4 E2M1 weights, FP8 E4M3 block scales, FP32 global scale; the
