@@ -76,13 +76,14 @@ def quantize_int4_asym(W, group=INT4_GROUP):
     (Linear)" (that page's quantizer is the symmetric one, zero-point 0).
 
     Per row n and group j of ``group`` consecutive k:
-      lo = min(0, min W),  hi = max(0, max W);  s = bf16(f32((hi - lo) / 15));
+      lo = min(0, min W),  hi = max(0, max W);  s = bf16(f32(f32(hi - lo) / 15));
       z = clamp(RNE(f32(-lo / s)), 0, 15);
       code = clamp(RNE(f32(W / s)) + z, 0, 15)  (unsigned);
       dequantized weight (code - z) * s;  a group with s == 0 has codes 0, z 0.
     Readings (no page gives them): the range includes 0 so that zero is
     exactly representable, the scale is bf16 like the symmetric format's,
-    the zero point an integer in [0, 15].
+    the zero point an integer in [0, 15], and the range is formed in fp32
+    before the division (the order of the fp32 operations is fixed here).
 
     Returns (codes uint8 [N, K], scale bits uint16 [N, K/group], zero points
     uint8 [N, K/group]).
@@ -94,7 +95,7 @@ def quantize_int4_asym(W, group=INT4_GROUP):
     B = _blocks(W, group)
     lo = np.minimum(B.min(axis=2), 0.0)
     hi = np.maximum(B.max(axis=2), 0.0)
-    s = bf16(f32((hi - lo) / 15.0))
+    s = bf16(f32(f32(hi - lo) / 15.0))
     safe = np.where(s > 0, s, 1.0)
     z = np.clip(np.rint(f32(-lo / safe)), 0, 15)
     z = np.where(s > 0, z, 0.0)
