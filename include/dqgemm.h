@@ -56,13 +56,21 @@ extern "C" {
  *   DQ_FP8_STATIC  as DQ_FP8_WO, plus global_scale = the calibrated fp32
  *                  per-tensor activation scale s_x; the GEMM runs FP8 x FP8
  *                  on e4m3(x / s_x) and rescales by s_x * s_w[n].
+ *   DQ_INT4_ASYM_G128  asymmetric INT4 with a zero point per group of 128
+ *                  (the zero-point counterpart of the INT4 page's symmetric
+ *                  format): packed u8 [N, K/2] unsigned nibbles 0..15, low
+ *                  nibble = even k; scales u8 [3 * N * K/128]: the bf16
+ *                  scales [N, K/128] followed by the u8 zero points
+ *                  [N, K/128] in [0, 15]; weight = (code - z) * s;
+ *                  K % 128 == 0
  */
 typedef enum {
   DQ_INT4_G128 = 0,
   DQ_NVFP4 = 1,
   DQ_MXFP4 = 2,
   DQ_FP8_WO = 3,
-  DQ_FP8_STATIC = 4
+  DQ_FP8_STATIC = 4,
+  DQ_INT4_ASYM_G128 = 5
 } dqgemm_format;
 
 typedef enum {
@@ -135,6 +143,9 @@ dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x,
  *   MXFP4  e = floor(log2 amax_blk32) - 2 in [-127,127]; code e+127 (0 for a
  *          zero block); c = e2m1(W * 2^-e), saturating
  *   FP8    s[n] = max|W[n,:]|/448; c = e4m3(W/s[n]) (0 for a zero row)
+ *   INT4 asymmetric  lo = min(0, min W), hi = max(0, max W) per group;
+ *          s = bf16(f32(hi - lo)/15); z = clamp(rne(-lo/s), 0, 15);
+ *          c = clamp(rne(W/s) + z, 0, 15); s == 0 -> c = 0, z = 0
  * `global_scale` (host, may be NULL) receives g for NVFP4 and 1 otherwise.
  * DQ_ERR_INVALID_ARG if W holds a non-finite value. */
 dqgemm_status dqgemm_pack_host(dqgemm_format fmt, const float* W, int K, int N,

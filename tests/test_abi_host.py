@@ -45,7 +45,7 @@ def _weights(N, K, seed, kind="uniform"):
     return W.astype(np.float32)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4", "fp8"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4", "fp8", "int4_asym"])
 @pytest.mark.parametrize("kind", ["uniform", "wide"])
 def test_pack_host_is_bit_identical_to_oracle(fmt, kind):
     N, K = 96, 512
@@ -67,7 +67,8 @@ def test_pack_host_hand_example_int4():
 
 
 @pytest.mark.parametrize("fmt,K,N", [("int4", 100, 8), ("nvfp4", 24, 16), ("nvfp4", 32, 8),
-                                     ("mxfp4", 48, 32), ("mxfp4", 64, 16), ("fp8", 8, 4), ("int4", 0, 8)])
+                                     ("mxfp4", 48, 32), ("mxfp4", 64, 16), ("fp8", 8, 4), ("int4", 0, 8),
+                                     ("int4_asym", 200, 8)])
 def test_pack_host_rejects_bad_shapes(fmt, K, N):
     W = np.zeros((max(N, 1), max(K, 1)), np.float32)
     st = dq._native.lib().dqgemm_pack_host(dq.FORMATS[fmt], W.ctypes.data, K, N, W.ctypes.data, W.ctypes.data, None)

@@ -19,7 +19,7 @@ from gpu_util import (bf16_values, check_close, dev, make_layer, run, scales_ten
 
 pytestmark = pytest.mark.gpu
 
-WO_FORMATS = ["int4", "nvfp4", "mxfp4", "fp8"]
+WO_FORMATS = ["int4", "nvfp4", "mxfp4", "fp8", "int4_asym"]
 ALL_FORMATS = WO_FORMATS + ["fp8_static"]
 
 
@@ -62,7 +62,7 @@ def test_pack_device_bit_identical_to_oracle(fmt, N, K):
 def test_dequantize_bit_exact(fmt, N, K, kind):
     if fmt in ("nvfp4", "mxfp4") and N % 32:
         N = 224
-    if fmt == "int4" and K % 128:
+    if fmt in ("int4", "int4_asym") and K % 128:
         K = 384
     if fmt == "mxfp4" and K % 32:
         K = 288
@@ -117,7 +117,7 @@ def test_gemm_matches_oracle(fmt, M, K, N):
         dq.dqgemm_destroy(h)
 
 
-@pytest.mark.parametrize("fmt,K,N", [("int4", 384, 200), ("fp8", 400, 136), ("nvfp4", 272, 176),
+@pytest.mark.parametrize("fmt,K,N", [("int4", 384, 200), ("int4_asym", 640, 136), ("fp8", 400, 136), ("nvfp4", 272, 176),
                                      ("mxfp4", 288, 160), ("fp8_static", 208, 72)])
 @pytest.mark.parametrize("M", [5, 40])
 def test_gemm_ragged_k_and_n(fmt, K, N, M):

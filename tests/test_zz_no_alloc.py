@@ -39,7 +39,7 @@ def _pack(entry, fmt, W):
     return packed.cpu().numpy(), scales.cpu().numpy().view(np.uint8), g
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "fp8"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "fp8", "int4_asym"])
 def test_noalloc_packer_matches_the_allocating_packer_on_two_calls(fmt):
     # the second call has a 1000x smaller tensor amax: a stale maximum left in
     # the shared scratch by the first call would change its global scale

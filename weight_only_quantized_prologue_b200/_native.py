@@ -14,7 +14,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdqgemm.so")
 
-FORMATS = {"int4": 0, "nvfp4": 1, "mxfp4": 2, "fp8": 3, "fp8_static": 4}
+FORMATS = {"int4": 0, "nvfp4": 1, "mxfp4": 2, "fp8": 3, "fp8_static": 4, "int4_asym": 5}
 STATUS_NAMES = {0: "DQ_OK", 1: "DQ_ERR_INVALID_ARG", 2: "DQ_ERR_UNSUPPORTED", 3: "DQ_ERR_ALIGNMENT",
                 4: "DQ_ERR_ALLOC", 5: "DQ_ERR_CUDA", 6: "DQ_ERR_TIMEOUT"}
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_ALIGNMENT = 0, 1, 2, 3
@@ -98,6 +98,8 @@ def storage_shapes(fmt, K, N):
     """Canonical (packed shape, packed dtype, scales shape, scales dtype) of a format."""
     if fmt == "int4":
         return (N, K // 2), np.uint8, (N, K // 128), np.uint16
+    if fmt == "int4_asym":   # bf16 scales [N, K/128] then u8 zero points [N, K/128], one buffer
+        return (N, K // 2), np.uint8, (3 * N * (K // 128),), np.uint8
     if fmt == "nvfp4":
         return (N, K // 2), np.uint8, (N, K // 16), np.uint8
     if fmt == "mxfp4":

@@ -59,6 +59,7 @@ size_t packed_bytes(int fmt, int K, int N) { return is_4bit(fmt) ? (size_t)N * K
 size_t scale_bytes(int fmt, int K, int N) {
   switch (fmt) {
     case FMT_INT4: return (size_t)N * (K / 128) * 2;
+    case FMT_INT4A: return (size_t)N * (K / 128) * 3;   // bf16 scales, then u8 zero points
     case FMT_NVFP4: return (size_t)N * (K / 16);
     case FMT_MXFP4: return (size_t)N * (K / 32);
     default: return (size_t)N * 4;
@@ -66,9 +67,10 @@ size_t scale_bytes(int fmt, int K, int N) {
 }
 
 dqgemm_status check_shape(int fmt, int K, int N) {
-  if (fmt < 0 || fmt > 4 || K <= 0 || N <= 0) return DQ_ERR_INVALID_ARG;
+  if (fmt < 0 || fmt > FMT_INT4A || K <= 0 || N <= 0) return DQ_ERR_INVALID_ARG;
   switch (fmt) {
-    case FMT_INT4: return K % 128 ? DQ_ERR_INVALID_ARG : DQ_OK;
+    case FMT_INT4:
+    case FMT_INT4A: return K % 128 ? DQ_ERR_INVALID_ARG : DQ_OK;
     case FMT_NVFP4: return (K % 16 || N % 16) ? DQ_ERR_INVALID_ARG : DQ_OK;
     case FMT_MXFP4: return (K % 32 || N % 32) ? DQ_ERR_INVALID_ARG : DQ_OK;
     default: return K % 16 ? DQ_ERR_INVALID_ARG : DQ_OK;
@@ -103,7 +105,7 @@ void relayout(int fmt, int K, int N, int KS, int NT, const std::vector<uint8_t>&
                 const int k0 = s * STAGE_K + 64 * h + 32 * j + 8 * w;
                 uint32_t c[8], word = 0;
                 for (int i = 0; i < 8; ++i) c[i] = nib(n, k0 + i);
-                if (fmt == FMT_INT4) {
+                if (fmt == FMT_INT4 || fmt == FMT_INT4A) {
                   for (int jj = 0; jj < 4; ++jj) word |= (c[2 * jj] << (4 * jj)) | (c[2 * jj + 1] << (16 + 4 * jj));
                 } else {
                   uint32_t m[8], sg[8];
@@ -116,11 +118,13 @@ void relayout(int fmt, int K, int N, int KS, int NT, const std::vector<uint8_t>&
                 put32(ch + ((h * 2 + j) * TILE_N + r) * 16 + w * 4, word);
               }
           uint8_t* sc = ch + PACKED4_BYTES;
-          if (fmt == FMT_INT4) {
+          if (fmt == FMT_INT4 || fmt == FMT_INT4A) {
             const int groups = K / 128;
             uint16_t v = 0;
             if (n < N && s < groups) std::memcpy(&v, &scales[((size_t)n * groups + s) * 2], 2);
             std::memcpy(sc + r * 2, &v, 2);
+            if (fmt == FMT_INT4A)
+              sc[TILE_N * 2 + r] = (n < N && s < groups) ? scales[(size_t)2 * N * groups + (size_t)n * groups + s] : 0;
           } else if (fmt == FMT_NVFP4) {
             const int blocks = K / 16;
             for (int h = 0; h < 2; ++h)
@@ -328,6 +332,7 @@ int max_clusters_fmt(int bn, int split) {
 #define DQ_FMT_SWITCH(fmt, CALL)                  \
   switch (fmt) {                                  \
     case FMT_INT4: { constexpr int F = FMT_INT4; CALL; } break;   \
+    case FMT_INT4A: { constexpr int F = FMT_INT4A; CALL; } break; \
     case FMT_NVFP4: { constexpr int F = FMT_NVFP4; CALL; } break; \
     case FMT_MXFP4: { constexpr int F = FMT_MXFP4; CALL; } break; \
     case FMT_FP8: { constexpr int F = FMT_FP8; CALL; } break;     \
@@ -589,6 +594,19 @@ dqgemm_status dqgemm_pack_host(dqgemm_format fmt_, const float* W, int K, int N,
         for (int i = 0; i < 64; ++i)
           P[(size_t)n * (K / 2) + gi * 64 + i] = (uint8_t)((c8[2 * i] & 0xF) | ((c8[2 * i + 1] & 0xF) << 4));
       }
+    } else if (fmt == FMT_INT4A) {
+      uint8_t* S = static_cast<uint8_t*>(scales);
+      const size_t G = (size_t)N * (K / 128);
+      for (int gi = 0; gi < K / 128; ++gi) {
+        const size_t idx = (size_t)n * (K / 128) + gi;
+        uint8_t z = 0;
+        const uint16_t sb = quant_int4_asym_group(w + gi * 128, 128, cu.data(), &z);
+        S[idx * 2] = (uint8_t)(sb & 0xFF);
+        S[idx * 2 + 1] = (uint8_t)(sb >> 8);
+        S[2 * G + idx] = z;
+        for (int i = 0; i < 64; ++i)
+          P[(size_t)n * (K / 2) + gi * 64 + i] = (uint8_t)(cu[2 * i] | (cu[2 * i + 1] << 4));
+      }
     } else if (fmt == FMT_NVFP4) {
       g = nvfp4_global_scale(amax);
       uint8_t* S = static_cast<uint8_t*>(scales);
@@ -631,6 +649,9 @@ dqgemm_status dqgemm_pack_device(dqgemm_format fmt_, const float* W, int K, int 
   if (fmt == FMT_INT4) {
     const long long n = (long long)N * (K / 128);
     pack_int4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint16_t*>(scales));
+  } else if (fmt == FMT_INT4A) {
+    const long long n = (long long)N * (K / 128);
+    pack_int4a_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint8_t*>(scales));
   } else if (fmt == FMT_NVFP4) {
     amax_kernel<<<(unsigned)std::min<long long>((count + T - 1) / T, 4096), T, 0, s>>>(W, count, amax);
     const long long n = (long long)N * (K / 16);
@@ -708,6 +729,9 @@ dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt_, const float* W, int
   if (fmt == FMT_INT4) {
     const long long n = (long long)N * (K / 128);
     pack_int4_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint16_t*>(scales));
+  } else if (fmt == FMT_INT4A) {
+    const long long n = (long long)N * (K / 128);
+    pack_int4a_kernel<<<(unsigned)((n + T - 1) / T), T, 0, s>>>(W, N, K, P, static_cast<uint8_t*>(scales));
   } else if (fmt == FMT_NVFP4) {
     float* scratch = noalloc_scratch(&st);
     if (!scratch) return st;

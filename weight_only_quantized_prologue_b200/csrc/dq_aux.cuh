@@ -75,6 +75,23 @@ __global__ void pack_int4_kernel(const float* W, int N, int K, uint8_t* packed, 
   for (int i = 0; i < 64; ++i) dst[i] = (uint8_t)((c[2 * i] & 0xF) | ((c[2 * i + 1] & 0xF) << 4));
 }
 
+// asymmetric INT4: scales bf16 [N, K/128] then zero points u8 [N, K/128],
+// one buffer (the canonical storage)
+__global__ void pack_int4a_kernel(const float* W, int N, int K, uint8_t* packed, uint8_t* scales) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int groups = K / 128;
+  const long long G = (long long)N * groups;
+  if (gid >= G) return;
+  const int n = (int)(gid / groups), g = (int)(gid % groups);
+  uint8_t c[128], z;
+  const uint16_t sb = quant_int4_asym_group(W + (size_t)n * K + g * 128, 128, c, &z);
+  scales[gid * 2] = (uint8_t)(sb & 0xFF);
+  scales[gid * 2 + 1] = (uint8_t)(sb >> 8);
+  scales[2 * G + gid] = z;
+  uint8_t* dst = packed + (size_t)n * (K / 2) + g * 64;
+  for (int i = 0; i < 64; ++i) dst[i] = (uint8_t)((c[2 * i] & 0xF) | ((c[2 * i + 1] & 0xF) << 4));
+}
+
 __global__ void amax_kernel(const float* W, long long count, unsigned int* amax_bits) {
   float a = 0.f;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;

@@ -135,6 +135,32 @@ DQ_HD uint16_t quant_int4_group(const float* w, int n, int8_t* codes) {
   return sb;
 }
 
+// INT4 asymmetric: lo = min(0, min w), hi = max(0, max w),
+// s = bf16((hi - lo)/15), z = clamp(rne(-lo/s), 0, 15),
+// c = clamp(rne(w/s) + z, 0, 15) (unsigned); a group with s == 0 has codes
+// 0 and z 0.  Writes n codes and *zero, returns the scale's bf16 bits.
+DQ_HD uint16_t quant_int4_asym_group(const float* w, int n, uint8_t* codes, uint8_t* zero) {
+  float lo = 0.f, hi = 0.f;
+  for (int i = 0; i < n; ++i) {
+    lo = fminf(lo, w[i]);
+    hi = fmaxf(hi, w[i]);
+  }
+  const uint16_t sb = bf16_bits_rn(fdiv(hi - lo, 15.f));
+  const float s = bf16_to_f(sb);
+  float z = 0.f;
+  if (s > 0.f) {
+    z = frint(fdiv(-lo, s));
+    z = z < 0.f ? 0.f : (z > 15.f ? 15.f : z);
+  }
+  for (int i = 0; i < n; ++i) {
+    float q = s > 0.f ? frint(fdiv(w[i], s)) + z : 0.f;
+    q = q < 0.f ? 0.f : (q > 15.f ? 15.f : q);
+    codes[i] = (uint8_t)q;
+  }
+  *zero = (uint8_t)z;
+  return sb;
+}
+
 DQ_HD float nvfp4_global_scale(float amax) { return amax > 0.f ? fdiv(amax, 2688.f) : 1.f; }
 
 // NVFP4 block of 16: sb = e4m3((amax/6)/g), c = e2m1(w / (dec(sb)*g)).

@@ -326,6 +326,17 @@ __device__ __forceinline__ void unpack_int4(uint32_t q, uint32_t s2, uint32_t* o
   }
 }
 
+// Unsigned INT4 (asymmetric format): 0x4300 | u is the bf16 of 128 + u, and
+// zs2 holds bf16(128 + z) twice, so one sub and one mul give (u - z) * s
+// exactly.
+__device__ __forceinline__ void unpack_int4u(uint32_t q, uint32_t zs2, uint32_t s2, uint32_t* o) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+    o[j] = bmul2(bsub2(v, zs2), s2);
+  }
+}
+
 // E2M1: magnitude bits (e1 e0 m) placed at bf16 bits 8..6 with the sign at
 // bit 15 read as a bf16 are exactly e2m1 * 2^-126 (the subnormal code 0.5
 // lands on a bf16 subnormal, code 0 on zero).  The block scale word s2

@@ -157,9 +157,14 @@ __device__ __forceinline__ void prologue_half(const uint8_t* chunk, int r, int h
     const uint4 v = lds128(chunk + ((h * 2 + hp) * TILE_N + r) * 16);
     const uint8_t* sc = chunk + PACKED4_BYTES;
     uint32_t sa, sb;   // bf16x2 scale words of the two 8-word halves of v
-    if constexpr (FMT == FMT_INT4) {
+    uint32_t zs2 = 0;   // asymmetric INT4: bf16(128 + z) twice
+    if constexpr (FMT == FMT_INT4 || FMT == FMT_INT4A) {
       const uint32_t s = *reinterpret_cast<const uint16_t*>(sc + r * 2);
       sa = sb = s | (s << 16);
+      if constexpr (FMT == FMT_INT4A) {
+        const uint32_t zs = 0x4300u | sc[TILE_N * 2 + r];
+        zs2 = zs | (zs << 16);
+      }
     } else if constexpr (FMT == FMT_NVFP4) {
       const uint32_t c2 = *reinterpret_cast<const uint16_t*>(sc + (h * TILE_N + r) * 4 + hp * 2);
       const uint32_t a = nvfp4_scale_bf16(c2 & 0xFFu), b = nvfp4_scale_bf16(c2 >> 8);
@@ -175,6 +180,11 @@ __device__ __forceinline__ void prologue_half(const uint8_t* chunk, int r, int h
       unpack_int4(v.y, sa, o + 4);
       unpack_int4(v.z, sb, o + 8);
       unpack_int4(v.w, sb, o + 12);
+    } else if constexpr (FMT == FMT_INT4A) {
+      unpack_int4u(v.x, zs2, sa, o + 0);
+      unpack_int4u(v.y, zs2, sa, o + 4);
+      unpack_int4u(v.z, zs2, sb, o + 8);
+      unpack_int4u(v.w, zs2, sb, o + 12);
     } else {
       unpack_e2m1(v.x, sa, o + 0);
       unpack_e2m1(v.y, sa, o + 4);

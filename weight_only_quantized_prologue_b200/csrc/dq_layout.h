@@ -20,6 +20,7 @@
 // each bf16x2 operand pair comes out with one shift and one mask (see
 // dq_common.cuh for the extraction):
 //   INT4 nibbles n0..n7:  n_{2j} at bits 4j..4j+3, n_{2j+1} at 16+4j..16+4j+3
+//                         (the same for the unsigned codes of asymmetric INT4)
 //   E2M1 (NVFP4/MXFP4) magnitude c = n & 7 and sign s = n >> 3:
 //        c0@0  c1@16 s0@14 s1@30 | c2@3 c3@19 s2@12 s3@28 |
 //        c4@6  c5@22 s4@15 s5@31 | c6@9 c7@25 s6@13 s7@29
@@ -27,6 +28,7 @@
 //        m0@0 m1@16 s0@15 s1@31 | m2@7 m3@23 s2@14 s3@30
 // Scales follow the 8192 packed bytes of a 4-bit chunk:
 //   INT4   bf16 s[r] for the group of this stage        (128 x 2 B)
+//   INT4 asymmetric  bf16 s[r] as INT4, then the zero point z[r] (128 x 1 B)
 //   NVFP4  E4M3 codes of blocks 4h..4h+3 at (h*128 + r)*4 (2 x 128 x 4 B)
 //   MXFP4  E8M0 codes of blocks 2h..2h+1 at (h*128 + r)*2 (2 x 128 x 2 B)
 // FP8 weight-only chunks hold codes only (the per-channel scale is applied
@@ -40,9 +42,10 @@
 namespace dq {
 
 enum Fmt { FMT_INT4 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_FP8S = 4,
+           FMT_INT4A = 5,   // asymmetric INT4, per-group zero point
            // static FP8 GEMM fed with activations quantized beforehand (same
            // weight chunks as FMT_FP8S; a kernel variant, not a storage format)
-           FMT_FP8SQ = 5 };
+           FMT_FP8SQ = 8 };
 
 constexpr int TILE_N = 128;      // output channels per tile (MMA M)
 constexpr int STAGE_K = 128;     // k per pipeline stage (= one INT4 group)
@@ -50,13 +53,14 @@ constexpr int PACKED4_BYTES = TILE_N * STAGE_K / 2;   // 8192
 
 __host__ __device__ constexpr int chunk_bytes(int fmt) {
   return fmt == FMT_INT4 ? PACKED4_BYTES + TILE_N * 2
+       : fmt == FMT_INT4A ? PACKED4_BYTES + TILE_N * 3
        : fmt == FMT_NVFP4 ? PACKED4_BYTES + TILE_N * 8
        : fmt == FMT_MXFP4 ? PACKED4_BYTES + TILE_N * 4
        : TILE_N * STAGE_K;
 }
 
 __host__ __device__ constexpr bool is_4bit(int fmt) {
-  return fmt == FMT_INT4 || fmt == FMT_NVFP4 || fmt == FMT_MXFP4;
+  return fmt == FMT_INT4 || fmt == FMT_INT4A || fmt == FMT_NVFP4 || fmt == FMT_MXFP4;
 }
 
 }  // namespace dq

@@ -19,7 +19,7 @@ import torch
 
 from . import QuantizedLinear
 
-FORMATS = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static")
+FORMATS = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static", "int4_asym")
 
 # live layers by handle value, so the op can reach the Python object (the
 # static-FP8 path needs its activation scale and K)
