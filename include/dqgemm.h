@@ -118,6 +118,22 @@ dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* s
  * this is faster.  DQ_ERR_UNSUPPORTED for other formats. */
 dqgemm_status dqgemm_run_fp8_static_quantized(dqgemm_handle h, const void* q, int M, void* y, void* stream);
 
+/* Chained static FP8 (the static page's two-layer "Graph after export", where
+ * the next layer's Q node reads this layer's output): as dqgemm_run, but the
+ * result leaves the kernel as the next layer's e4m3 activation codes,
+ * q_out[m, n] = e4m3(f32(y[m, n]) / s_out) with y the bf16 result, IEEE
+ * division, round to nearest even, saturating -- the codes
+ * dqgemm_quantize_act_fp8(y, s_out) would give.  q_out: device u8 [M, N],
+ * 16-byte aligned; s_out > 0 (DQ_ERR_INVALID_ARG otherwise).  Any format. */
+dqgemm_status dqgemm_run_quantized_out(dqgemm_handle h, const void* x, int M, void* q_out, float s_out,
+                                       void* stream);
+
+/* DQ_FP8_STATIC only: both ends quantized -- the input as for
+ * dqgemm_run_fp8_static_quantized, the output as for
+ * dqgemm_run_quantized_out (a middle layer of a static-FP8 chain). */
+dqgemm_status dqgemm_run_fp8_static_quantized_out(dqgemm_handle h, const void* q, int M, void* q_out,
+                                                  float s_out, void* stream);
+
 /* Release the handle and its device memory (synchronizes the device). */
 dqgemm_status dqgemm_destroy(dqgemm_handle h);
 

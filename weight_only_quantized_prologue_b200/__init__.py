@@ -25,6 +25,8 @@ from ._native import (  # noqa: F401
     dqgemm_quantize_act_fp8,
     dqgemm_run,
     dqgemm_run_fp8_static_quantized,
+    dqgemm_run_fp8_static_quantized_out,
+    dqgemm_run_quantized_out,
     dqgemm_selftest_timeout,
     dqgemm_status_string,
     storage_shapes,
@@ -75,6 +77,33 @@ class QuantizedLinear:
             dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)
         else:
             dqgemm_run(self._h, x, M, out, stream)
+        return out
+
+    def quantized_out(self, x, s_out, out=None, stream=None):
+        """The layer with its result leaving as the next static-FP8 layer's
+        e4m3 codes, e4m3(f32(y) / s_out) (uint8 [M, N]); x as for __call__."""
+        import torch
+
+        M = x.shape[0]
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.uint8, device=x.device)
+        if self.fmt == "fp8_static" and M >= self.STATIC_PREQUANT_M:
+            q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
+            dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
+            dqgemm_run_fp8_static_quantized_out(self._h, q, M, out, s_out, stream)
+        else:
+            dqgemm_run_quantized_out(self._h, x, M, out, s_out, stream)
+        return out
+
+    def from_codes(self, q, out=None, stream=None):
+        """Static FP8 only: the layer on activations already quantized with
+        its own scale (uint8 e4m3 codes [M, K], e.g. from quantized_out)."""
+        import torch
+
+        M = q.shape[0]
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=q.device)
+        dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)
         return out
 
     def dequantize(self, stream=None):

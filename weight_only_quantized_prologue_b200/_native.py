@@ -42,6 +42,8 @@ _SIGNATURES = {
     "dqgemm_create": [ctypes.POINTER(_VP), _I, _I, _I, _VP, _VP, _F, _VP],
     "dqgemm_run": [_VP, _VP, _I, _VP, _VP],
     "dqgemm_run_fp8_static_quantized": [_VP, _VP, _I, _VP, _VP],
+    "dqgemm_run_quantized_out": [_VP, _VP, _I, _VP, _F, _VP],
+    "dqgemm_run_fp8_static_quantized_out": [_VP, _VP, _I, _VP, _F, _VP],
     "dqgemm_destroy": [_VP],
     "dqgemm_dequantize": [_VP, _VP, _VP],
     "dqgemm_quantize_act_fp8": [_VP, _I, _I, _F, _VP, _VP],
@@ -126,6 +128,16 @@ def dqgemm_run(h, x, M, y, stream=None):
 def dqgemm_run_fp8_static_quantized(h, q, M, y, stream=None):
     _check(lib().dqgemm_run_fp8_static_quantized(h, _ptr(q), int(M), _ptr(y), _stream(stream)),
            "dqgemm_run_fp8_static_quantized")
+
+
+def dqgemm_run_quantized_out(h, x, M, q_out, s_out, stream=None):
+    _check(lib().dqgemm_run_quantized_out(h, _ptr(x), int(M), _ptr(q_out), float(s_out), _stream(stream)),
+           "dqgemm_run_quantized_out")
+
+
+def dqgemm_run_fp8_static_quantized_out(h, q, M, q_out, s_out, stream=None):
+    _check(lib().dqgemm_run_fp8_static_quantized_out(h, _ptr(q), int(M), _ptr(q_out), float(s_out),
+                                                      _stream(stream)), "dqgemm_run_fp8_static_quantized_out")
 
 
 def dqgemm_destroy(h):

@@ -232,11 +232,18 @@ template <int FMT, int BN>
 struct GemmLauncher {
   using C = GemmCfg<FMT, BN>;
   static cudaError_t set_attr() {
-    cudaError_t e = cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = set_attr_q<false>();
+    if (e == cudaSuccess) e = set_attr_q<true>();
+    return e;
+  }
+  template <bool QOUT>
+  static cudaError_t set_attr_q() {
+    cudaError_t e =
+        cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN, QOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     // every GEMM kernel asks for the same (largest) shared-memory carveout, so
     // back-to-back calls never reconfigure the SM's L1 / shared split
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN>, cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(dq_gemm_kernel<FMT, BN, QOUT>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     return e;
   }
@@ -266,7 +273,8 @@ struct GemmLauncher {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attrs[2];
     config(cfg, attrs, grid, p.split, st);
-    return cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN>, tm, p);
+    return p.yq ? cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, true>, tm, p)
+                : cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, false>, tm, p);
   }
   static int max_active_clusters(int split) {
     cudaLaunchConfig_t cfg;
@@ -274,7 +282,7 @@ struct GemmLauncher {
     config(cfg, attrs, split, split, nullptr);
     int n = 0;
     if (split > 1) {
-      if (cudaOccupancyMaxActiveClusters(&n, dq_gemm_kernel<FMT, BN>, &cfg) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveClusters(&n, dq_gemm_kernel<FMT, BN, false>, &cfg) != cudaSuccess) {
         cudaGetLastError();
         n = 0;
       }
@@ -503,8 +511,10 @@ dqgemm_status dqgemm_get_plan(dqgemm_handle h, int M, dqgemm_plan* plan) {
   return DQ_OK;
 }
 
-static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, void* y, void* stream) {
+static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, void* y, bool yq, float s_out,
+                              void* stream) {
   if (!h || !x || !y || M < 1) return DQ_ERR_INVALID_ARG;
+  if (yq && !(std::isfinite(s_out) && s_out > 0.f)) return DQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
   dqgemm_plan pl;
   fill_plan(h, M, &pl);
@@ -515,7 +525,9 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   p.wchunks = h->wchunks;
   p.col_scale = h->col_scale;
   p.bias = h->bias;
-  p.y = static_cast<__nv_bfloat16*>(y);
+  p.y = yq ? nullptr : static_cast<__nv_bfloat16*>(y);
+  p.yq = yq ? static_cast<uint8_t*>(y) : nullptr;
+  p.s_out = yq ? s_out : 1.f;
   p.status = h->status;
   p.sigma = h->sigma;
   p.s_x = h->s_x;
@@ -539,13 +551,25 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
 }
 
 dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream) {
-  return run_gemm(h, x, false, M, y, stream);
+  return run_gemm(h, x, false, M, y, false, 1.f, stream);
 }
 
 dqgemm_status dqgemm_run_fp8_static_quantized(dqgemm_handle h, const void* q, int M, void* y, void* stream) {
   if (!h) return DQ_ERR_INVALID_ARG;
   if (h->fmt != FMT_FP8S) return DQ_ERR_UNSUPPORTED;
-  return run_gemm(h, q, true, M, y, stream);
+  return run_gemm(h, q, true, M, y, false, 1.f, stream);
+}
+
+dqgemm_status dqgemm_run_quantized_out(dqgemm_handle h, const void* x, int M, void* q_out, float s_out,
+                                       void* stream) {
+  return run_gemm(h, x, false, M, q_out, true, s_out, stream);
+}
+
+dqgemm_status dqgemm_run_fp8_static_quantized_out(dqgemm_handle h, const void* q, int M, void* q_out,
+                                                  float s_out, void* stream) {
+  if (!h) return DQ_ERR_INVALID_ARG;
+  if (h->fmt != FMT_FP8S) return DQ_ERR_UNSUPPORTED;
+  return run_gemm(h, q, true, M, q_out, true, s_out, stream);
 }
 
 dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream) {

@@ -54,10 +54,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* wchunks, co
 __global__ void act_quant_kernel(const __nv_bfloat16* x, long long count, float s_x, uint8_t* q) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
        i += (long long)gridDim.x * blockDim.x) {
-    const float v = __fdiv_rn(__bfloat162float(x[i]), s_x);
-    uint8_t c = (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
-    if ((c & 0x7F) == 0) c = signbit(v) ? 0x80 : 0x00;   // a zero keeps the sign of x
-    q[i] = c;
+    q[i] = e4m3_code(__fdiv_rn(__bfloat162float(x[i]), s_x));
   }
 }
 

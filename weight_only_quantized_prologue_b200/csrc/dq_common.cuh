@@ -195,6 +195,14 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank)
 }
 
 
+// e4m3 code of v, saturating to +-448, round to nearest even; a zero result
+// keeps the sign of v (static FP8 activation codes)
+__device__ __forceinline__ uint8_t e4m3_code(float v) {
+  uint8_t c = (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+  if ((c & 0x7F) == 0) c = signbit(v) ? 0x80 : 0x00;
+  return c;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -53,7 +53,16 @@ struct GemmParams {
   int split;                     // CTAs per tile (cluster size); 1 = whole tiles
   int x3d;                       // x map is 3-D {64, M, K/64}: one box per stage
   unsigned long long timeout_ns;
+  uint8_t* yq;                   // if set: y goes out as e4m3 codes of bf16(y) / s_out
+  float s_out;                   //   (the next static-FP8 layer's activation codes)
 };
+
+// the e4m3 code of an output for the next static-FP8 layer,
+// q = e4m3(f32(bf16(v)) / s_out): the code dqgemm_quantize_act_fp8 gives
+// for the bf16 output y = bf16(v)
+__device__ __forceinline__ uint8_t out_code(const GemmParams& p, float v) {
+  return e4m3_code(__fdiv_rn(__bfloat162float(__float2bfloat16_rn(v)), p.s_out));
+}
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
 __host__ __device__ constexpr int pow2_at_least(int v) {
@@ -227,7 +236,10 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
   }
 }
 
-template <int FMT, int BN>
+// QOUT: the output leaves as the next static-FP8 layer's e4m3 codes (a
+// separate instantiation, so the common bf16 epilogue stays as compact as
+// it can be)
+template <int FMT, int BN, bool QOUT>
 __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                          const GemmParams p) {
   using C = GemmCfg<FMT, BN>;
@@ -508,10 +520,18 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
         const float e_sig = epi[et], e_bias = epi[256 + et];
         if (n_row < p.N) {
+          if constexpr (!QOUT) {
 #pragma unroll
-          for (int i = 0; i < HALF; ++i) {
-            const int m = m_tile * BN + h * HALF + i;
-            if (m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(acc[i], e_sig, e_bias));
+            for (int i = 0; i < HALF; ++i) {
+              const int m = m_tile * BN + h * HALF + i;
+              if (m < p.M) p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(acc[i], e_sig, e_bias));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < HALF; ++i) {
+              const int m = m_tile * BN + h * HALF + i;
+              if (m < p.M) p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(acc[i], e_sig, e_bias));
+            }
           }
         }
       }
@@ -552,14 +572,26 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         v[i] = pr == q ? part[c * TILE_N + r] : ld_dsmem_f32(part + c * TILE_N + r, (uint32_t)pr);
       }
       float sum = 0.f;
+      if constexpr (!QOUT) {
 #pragma unroll
-      for (int i = 0; i < HALF; ++i) {
-        const int pr = i & (S - 1);
-        sum = pr == 0 ? v[i] : sum + v[i];
-        if (pr == S - 1) {
-          const int m = m_tile * BN + c0 + h + 2 * (i >> lg_s);
-          if (all_good && n_row < p.N && m < p.M)
-            p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
+        for (int i = 0; i < HALF; ++i) {
+          const int pr = i & (S - 1);
+          sum = pr == 0 ? v[i] : sum + v[i];
+          if (pr == S - 1) {
+            const int m = m_tile * BN + c0 + h + 2 * (i >> lg_s);
+            if (all_good && n_row < p.N && m < p.M)
+              p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          const int pr = i & (S - 1);
+          sum = pr == 0 ? v[i] : sum + v[i];
+          if (pr == S - 1) {
+            const int m = m_tile * BN + c0 + h + 2 * (i >> lg_s);
+            if (all_good && n_row < p.N && m < p.M) p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(sum, e_sig, e_bias));
+          }
         }
       }
     }
