@@ -48,15 +48,20 @@ WORKLOAD = ("Linear(3072->4096), x[32,3072] bf16, in INT4-g128 / NVFP4 / MXFP4 /
 
 
 def algorithmic_bytes(fmt, M, K, N, bias=True):
-    """Bytes one call must move: packed weight + scales (+ global scale) + x + y + bias."""
+    """Bytes one call must move: packed weight + scales (+ zero points, +
+    global scale) + x + y + bias."""
     if fmt == "int4":
         w = N * K // 2 + N * (K // 128) * 2
+    elif fmt == "int4_asym":
+        w = N * K // 2 + N * (K // 128) * 3
     elif fmt == "nvfp4":
         w = N * K // 2 + N * (K // 16) + 4
     elif fmt == "mxfp4":
         w = N * K // 2 + N * (K // 32)
-    else:
+    elif fmt in ("fp8", "fp8_static"):
         w = N * K + N * 4
+    else:
+        raise ValueError(f"unknown format {fmt!r}")
     return w + M * K * 2 + M * N * 2 + (N * 2 if bias else 0)
 
 
@@ -122,25 +127,33 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.out.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
-                    continue
-                for name, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(name)
+            lines = f.readlines()
         os.unlink(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return parse_clock_samples(lines)
+
+
+def parse_clock_samples(lines):
+    """Median SM clock, max SM clock and the throttle reasons seen in
+    `nvidia-smi --query-gpu=<ClockSampler.FIELDS> --format=csv,noheader,nounits`
+    output lines; None when no line parses."""
+    sm, mx, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx = float(parts[2])
+        except ValueError:
+            continue
+        for name, v in zip(names, parts[5:9]):
+            if v.lower().startswith("active"):
+                reasons.add(name)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
 # ---------------------------------------------------------------------------
@@ -586,7 +599,7 @@ def run_sweep(args):
     fmts = args.sweep_formats.split(",")
     for (K, N) in shapes:
         for fmt in fmts:
-            wb = algorithmic_bytes("fp8" if fmt == "fp8_static" else fmt, 0, K, N, bias=False)
+            wb = algorithmic_bytes(fmt, 0, K, N, bias=False)
             R = max(2, math.ceil(3 * l2 / wb))
             layers = []
             for r in range(R):
@@ -615,8 +628,7 @@ def run_sweep(args):
                     t1.record(stream)
                     t1.synchronize()
                 us = t0.elapsed_time(t1) * 1000.0 / reps
-                byts = algorithmic_bytes("fp8" if fmt == "fp8_static" else fmt, M, K, N,
-                                         bias=fmt != "fp8_static")
+                byts = algorithmic_bytes(fmt, M, K, N, bias=fmt != "fp8_static")
                 gbs = byts / (us * 1e-6) / 1e9
                 tflops = flops / (us * 1e-6) / 1e12
                 peak_t = peaks["bf16_tflops"] * (2.0 if fmt == "fp8_static" else 1.0)
