@@ -11,7 +11,8 @@ Modules
 formats   number formats: E2M1, E4M3 ("fn"), E8M0, BF16, FP32 rounding.
 quant     the weight quantizers and the nibble packer of the five formats.
 linear    dequantization, the fp64 GEMM reference, static-FP8 activation
-          quantization and calibration, SQNR.
+          quantization and calibration, SQNR, and the FP4 x FP4 reference
+          (dynamic MX / NVFP4 activation quantization).
 
 Parity status of every function is stated in its docstring; functions whose
 result is not pinned by an independent check say "parity unpinned".

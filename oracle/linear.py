@@ -9,6 +9,10 @@ Format names used here and by the tests:
   "mxfp4"      E2M1 + E8M0/32               (MXFP4 page)
   "fp8"        E4M3 + fp32 per channel      (FP8 weight-only page)
   "fp8_static" E4M3 weights and activations (static FP8 page)
+
+The FP4 x FP4 section at the end (dynamic activation quantization and the
+W4A4 reference) is the native-MMA variant the MXFP4 page names; the library
+has no kernel for it yet.
 """
 
 import numpy as np
@@ -206,3 +210,54 @@ def sqnr(a, b):
     b = np.asarray(b, dtype=np.float64).ravel()
     noise = max(np.linalg.norm(a - b), 1e-12)
     return 20.0 * np.log10(np.linalg.norm(a) / noise)
+
+
+# ---------------------------------------------------------------------------
+# FP4 x FP4 ("TorchAO MXFP4 Dynamic Activation + MX Weight (Linear)", intro:
+# the config is MX dynamic activation + MX weight, and native MXFP4 x MXFP4
+# needs B200).  Not served by the library yet; the reference of that path.
+# ---------------------------------------------------------------------------
+
+
+def quantize_act_mxfp4(x):
+    """Dynamic MX activation quantization: every row of x [M, K] (at its
+    bf16 value) is cut into blocks of 32 along K and quantized at call time
+    with the same recipe as the MX weight (shared exponent
+    floor(log2 amax) - 2, E2M1 elements).
+    Reading: "dynamic activation" means the scales come from the call's own
+    x, block by block along the reduction dimension, as for the weight.
+    Returns (codes uint8 [M, K], E8M0 scale codes uint8 [M, K/32]).
+    Parity: pinned by the MX weight pins (same quantizer) and by the
+    power-of-two and sign symmetries of the W4A4 tests."""
+    return quantize_mxfp4(np.asarray(x, dtype=np.float64))
+
+
+def quantize_act_nvfp4(x):
+    """Dynamic NVFP4 activation quantization: x [M, K] as one tensor through
+    the NVFP4 recipe (per-tensor fp32 global scale from amax(x), E4M3 scale
+    per block of 16 along K, E2M1 elements).
+    Reading: the pages pair NVFP4 only with BF16 activations; this is the
+    weight recipe applied to x unchanged, the global scale taken per call.
+    Returns (codes uint8 [M, K], E4M3 scale codes uint8 [M, K/16], g_x).
+    Parity: pinned as quantize_act_mxfp4."""
+    return quantize_nvfp4(np.asarray(x, dtype=np.float64))
+
+
+def w4a4_linear_ref(fmt, x, packed_w, scales_w, global_scale_w=1.0, bias=None):
+    """FP4 x FP4 Linear: y = sum_k deq(Q(x))[m, k] * deq(W)[n, k] + b[n], with
+    Q the dynamic activation quantizer of `fmt` ("mxfp4" or "nvfp4") and W in
+    the same format's storage.  Every dequantized operand is exact in fp64,
+    so this is the exact product of the two dequantized matrices plus the
+    bias; not rounded (the kernel rounds to bf16 once).
+    Parity: pinned by on-grid activations reducing to the weight-only
+    reference, brute force on a tiny case, and exact power-of-two and sign
+    symmetries."""
+    if fmt == "mxfp4":
+        cx, sx = quantize_act_mxfp4(x)
+        xd = e2m1_decode(cx) * np.repeat(e8m0_decode(sx), MXFP4_BLOCK, axis=1)
+    elif fmt == "nvfp4":
+        cx, sx, gx = quantize_act_nvfp4(x)
+        xd = e2m1_decode(cx) * np.repeat(e4m3_decode(sx), NVFP4_BLOCK, axis=1) * float(gx)
+    else:
+        raise ValueError(fmt)
+    return linear_ref(xd, dequant_exact(fmt, packed_w, scales_w, global_scale_w), bias)
