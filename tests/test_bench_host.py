@@ -89,3 +89,34 @@ def test_source_hash_tracks_csrc():
     h = bench.kernel_source_hash()
     assert len(h) == 16 and int(h, 16) >= 0
     assert h == bench.kernel_source_hash()
+
+
+def test_clock_sampler_with_fake_nvidia_smi(tmp_path, monkeypatch):
+    # the sampler process end to end, with a stand-in nvidia-smi that prints
+    # two samples and then idles until it is terminated
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\n"
+                    "echo '0, 1965, 1965, 600.0, 0x0, Not Active, Not Active, Not Active, Not Active'\n"
+                    "echo '0, 1935, 1965, 980.0, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "exec sleep 30\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ['PATH']}")
+    s = bench.ClockSampler(0)
+    s.start()
+    assert s.proc is not None
+    import time
+    deadline = time.time() + 10
+    while time.time() < deadline and os.path.getsize(s.path) == 0:
+        time.sleep(0.05)
+    time.sleep(0.2)
+    c = s.stop()
+    assert c == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    assert not os.path.exists(s.path)
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))
+    s = bench.ClockSampler(0)
+    s.start()
+    assert s.stop() is None
+    assert not os.path.exists(s.path)
