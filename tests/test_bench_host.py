@@ -120,3 +120,20 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     s.start()
     assert s.stop() is None
     assert not os.path.exists(s.path)
+
+
+def test_reference_arm_line():
+    # the reference arm times the oracle on the host cores; rank 0 alone
+    # prints, other ranks do no work
+    import argparse
+    from weight_only_quantized_prologue_b200 import synthetic  # noqa: F401
+
+    args = argparse.Namespace(steps=1, warmup=0)
+    assert bench.run_reference(args, rank=1, world=2) is None
+    res = bench.run_reference(args, rank=0, world=1)
+    assert res["impl"] == "reference" and res["dtype"] == "f64" and res["higher_is_better"] is False
+    assert res["value"] > 0 and res["unit"] == bench.UNIT and res["metric"] == bench.METRIC
+    assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["value"] == res["value"]
+    assert res["e2e"] == {"value": res["value"], "unit": res["unit"], "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+    json.dumps(res)
