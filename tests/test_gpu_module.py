@@ -58,3 +58,30 @@ def test_static_fp8_calibrate_then_quantize():
 def test_static_fp8_without_scales_is_refused():
     with pytest.raises(ValueError):
         M.quantize_(_model(3), "fp8_static")
+
+
+@pytest.mark.gpu
+def test_layer_rejects_bad_tensors_before_launch():
+    # wrong dtype / shape / layout never reach the kernel; an empty batch
+    # launches nothing and returns an empty result
+    torch.manual_seed(3)
+    w = torch.randn(128, 256, device="cuda") * 0.05
+    lin = dq.QuantizedLinear.from_float("int4", w.to(torch.bfloat16))    # bf16 weight: converted
+    x = synthetic.activations(8, 256, seed=1).cuda()
+    with pytest.raises(TypeError):
+        lin(x.float())
+    with pytest.raises(ValueError):
+        lin(x[:, :128])
+    with pytest.raises(ValueError):
+        lin(torch.empty(256, 8, dtype=torch.bfloat16, device="cuda").t())
+    with pytest.raises(ValueError):
+        lin(x, out=torch.empty(8, 64, dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        dq.QuantizedLinear("int4", 256, 128, torch.zeros(128, 100, dtype=torch.uint8, device="cuda"),
+                           torch.zeros(128, 2, dtype=torch.int16, device="cuda"))
+    y0 = lin(x[:0])
+    assert y0.shape == (0, 128)
+    y = lin(x)
+    torch.cuda.synchronize()
+    assert lin.last_error() == 0 and y.shape == (8, 128)
+    lin.close()

@@ -33,6 +33,29 @@ from ._native import (  # noqa: F401
 )
 
 
+def _require(t, name, shape=None, dtype=None, nbytes=None, device=None):
+    """Checks the library cannot make itself: its entry points take bare
+    device pointers, so a tensor of the wrong dtype, shape or layout would be
+    read or written out of bounds on the GPU."""
+    if not getattr(t, "is_cuda", False):
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if nbytes is not None and t.numel() * t.element_size() != nbytes:
+        raise ValueError(f"{name} must hold {nbytes} bytes, got {t.numel() * t.element_size()}")
+
+
+def _storage_bytes(fmt, K, N):
+    ps, pd, ss, sd = storage_shapes(fmt, K, N)
+    return (int(_np.prod(ps)) * _np.dtype(pd).itemsize, int(_np.prod(ss)) * _np.dtype(sd).itemsize)
+
+
 class QuantizedLinear:
     """One quantized Linear layer on the current CUDA device.
 
@@ -45,6 +68,16 @@ class QuantizedLinear:
     STATIC_PREQUANT_M = 128
 
     def __init__(self, fmt, K, N, packed, scales, global_scale=1.0, bias=None):
+        import torch
+
+        self._h = None
+        if fmt not in FORMATS:
+            raise ValueError(f"unknown format {fmt!r}; one of {tuple(FORMATS)}")
+        pb, sb = _storage_bytes(fmt, K, N)
+        _require(packed, "packed", nbytes=pb)
+        _require(scales, "scales", nbytes=sb, device=packed.device)
+        if bias is not None:
+            _require(bias, "bias", shape=(N,), dtype=torch.bfloat16, device=packed.device)
         self.fmt, self.K, self.N = fmt, K, N
         self.act_scale = float(global_scale) if fmt == "fp8_static" else None
         self._h = dqgemm_create(fmt, K, N, packed, scales, global_scale, bias)
@@ -55,22 +88,44 @@ class QuantizedLinear:
         layer.  ``act_scale`` is the static-FP8 per-tensor activation scale."""
         import torch
 
+        if not getattr(W, "is_cuda", False) or W.dim() != 2:
+            raise ValueError("W must be a 2-D CUDA tensor [N, K]")
+        W = W.detach().to(torch.float32).contiguous()
         N, K = W.shape
         ps, pd, ss, sd = storage_shapes(fmt, K, N)
         tdt = {_np.uint8: torch.uint8, _np.uint16: torch.int16, _np.float32: torch.float32}
         packed = torch.empty(ps, dtype=tdt[pd], device=W.device)
         scales = torch.empty(ss, dtype=tdt[sd], device=W.device)
-        g = dqgemm_pack_device("fp8" if fmt == "fp8_static" else fmt, W.contiguous(), packed, scales)
+        g = dqgemm_pack_device("fp8" if fmt == "fp8_static" else fmt, W, packed, scales)
         if fmt == "fp8_static":
             g = act_scale
         return cls(fmt, K, N, packed, scales, g, bias)
 
-    def __call__(self, x, out=None, stream=None):
+    def _check_x(self, x, dtype, name="x"):
         import torch
 
-        M = x.shape[0]
+        if getattr(x, "dim", lambda: 0)() != 2:
+            raise ValueError(f"{name} must be 2-D [M, {self.K}]")
+        _require(x, name, shape=(x.shape[0], self.K), dtype=dtype)
+        return x.shape[0]
+
+    def _out(self, out, M, dtype, device):
+        import torch
+
         if out is None:
-            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
+            return torch.empty((M, self.N), dtype=dtype, device=device)
+        _require(out, "out", shape=(M, self.N), dtype=dtype, device=device)
+        return out
+
+    def __call__(self, x, out=None, stream=None):
+        """y = x . deq(W)^T + b; x bf16 [M, K] contiguous on CUDA, y (``out``,
+        allocated if None) bf16 [M, N]."""
+        import torch
+
+        M = self._check_x(x, torch.bfloat16)
+        out = self._out(out, M, torch.bfloat16, x.device)
+        if M == 0:
+            return out
         if self.fmt == "fp8_static" and M >= self.STATIC_PREQUANT_M:
             q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
             dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
@@ -84,9 +139,10 @@ class QuantizedLinear:
         e4m3 codes, e4m3(f32(y) / s_out) (uint8 [M, N]); x as for __call__."""
         import torch
 
-        M = x.shape[0]
-        if out is None:
-            out = torch.empty((M, self.N), dtype=torch.uint8, device=x.device)
+        M = self._check_x(x, torch.bfloat16)
+        out = self._out(out, M, torch.uint8, x.device)
+        if M == 0:
+            return out
         if self.fmt == "fp8_static" and M >= self.STATIC_PREQUANT_M:
             q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
             dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
@@ -100,9 +156,12 @@ class QuantizedLinear:
         its own scale (uint8 e4m3 codes [M, K], e.g. from quantized_out)."""
         import torch
 
-        M = q.shape[0]
-        if out is None:
-            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=q.device)
+        if self.fmt != "fp8_static":
+            raise ValueError("from_codes needs a static FP8 layer")
+        M = self._check_x(q, torch.uint8, "q")
+        out = self._out(out, M, torch.bfloat16, q.device)
+        if M == 0:
+            return out
         dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)
         return out
 
