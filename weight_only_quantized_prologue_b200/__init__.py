@@ -51,6 +51,17 @@ def _require(t, name, shape=None, dtype=None, nbytes=None, device=None):
         raise ValueError(f"{name} must hold {nbytes} bytes, got {t.numel() * t.element_size()}")
 
 
+def _fits(t, cols, dtype, rows=None, device=None):
+    """Fast form of the _require checks for a 2-D operand [rows, cols]: True
+    exactly when _require(t, shape=(rows, cols), dtype, device) would pass."""
+    try:
+        return (t.dtype is dtype and t.is_cuda and t.dim() == 2 and t.shape[1] == cols
+                and (rows is None or t.shape[0] == rows) and t.is_contiguous()
+                and (device is None or t.device == device))
+    except AttributeError:
+        return False
+
+
 def _storage_bytes(fmt, K, N):
     ps, pd, ss, sd = storage_shapes(fmt, K, N)
     return (int(_np.prod(ps)) * _np.dtype(pd).itemsize, int(_np.prod(ss)) * _np.dtype(sd).itemsize)
@@ -102,19 +113,19 @@ class QuantizedLinear:
         return cls(fmt, K, N, packed, scales, g, bias)
 
     def _check_x(self, x, dtype, name="x"):
-        import torch
-
-        if getattr(x, "dim", lambda: 0)() != 2:
-            raise ValueError(f"{name} must be 2-D [M, {self.K}]")
-        _require(x, name, shape=(x.shape[0], self.K), dtype=dtype)
+        if not _fits(x, self.K, dtype):
+            if getattr(x, "dim", lambda: 0)() != 2:
+                raise ValueError(f"{name} must be 2-D [M, {self.K}]")
+            _require(x, name, shape=(x.shape[0], self.K), dtype=dtype)
         return x.shape[0]
 
     def _out(self, out, M, dtype, device):
-        import torch
-
         if out is None:
+            import torch
+
             return torch.empty((M, self.N), dtype=dtype, device=device)
-        _require(out, "out", shape=(M, self.N), dtype=dtype, device=device)
+        if not _fits(out, self.N, dtype, M, device):
+            _require(out, "out", shape=(M, self.N), dtype=dtype, device=device)
         return out
 
     def __call__(self, x, out=None, stream=None):
