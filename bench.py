@@ -304,6 +304,8 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         e2e_ms = aggregate_max(e2e_ms)
 
+    single = single_launch_us(torch, sets, stream)
+
     for s in sets:
         for l in list(s.layers.values()) + [s.mlp1, s.mlp2]:
             assert l.last_error() == 0, "device-side wait timed out"
@@ -339,8 +341,36 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps * CALLS_PER_STEP,
         "clocks": clocks,
+        "single_launch_us": single,
     }
     return result, sets
+
+
+def single_launch_us(torch, sets, stream, reps=8):
+    """Median device time of one call on its own: the stream is idle apart
+    from an L2 flush (a 256 MB memset) before it, so the call neither
+    overlaps a neighbour nor finds its weight in L2.  Per weight-only format;
+    None if the measurement itself fails (it is outside the timed step)."""
+    try:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        out = {}
+        with torch.cuda.stream(stream):
+            for f in LIN_FORMATS:
+                lat = []
+                for i in range(reps):
+                    st = sets[i % len(sets)]
+                    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    flush.zero_()
+                    a.record(stream)
+                    st.layers[f](st.x, out=st.y[f], stream=stream)
+                    z.record(stream)
+                    z.synchronize()
+                    lat.append(a.elapsed_time(z) * 1000.0)
+                out[f] = round(statistics.median(lat), 3)
+        del flush
+        return out
+    except Exception as e:      # noqa: BLE001 - report, do not lose the bench line
+        return {"error": str(e)[:200]}
 
 
 class EndToEnd:
@@ -458,7 +488,12 @@ class OracleWorkload:
         x, w, b = synthetic.linear_inputs(LM, LK, LN, seed=0)
         self.x = x.float().numpy().astype(np.float64)
         self.b = b.float().numpy().astype(np.float64)
-        self.store = {f: L.quantize_pack(f, w.numpy().astype(np.float64)) for f in LIN_FORMATS}
+        wv = w.numpy().astype(np.float64)
+        self.store, self.pack_s = {}, {}
+        for f in LIN_FORMATS:
+            t0 = time.perf_counter()
+            self.store[f] = L.quantize_pack(f, wv)
+            self.pack_s[f] = time.perf_counter() - t0
         w1, w2 = synthetic.mlp_weights(seed=7)
         w1v, w2v = w1.float().numpy().astype(np.float64), w2.float().numpy().astype(np.float64)
         cal = [synthetic.activations(LM, MLP_IN, seed=s).float().numpy().astype(np.float64) for s in range(1, 11)]
@@ -524,9 +559,23 @@ def cpu_baseline(synthetic, budget_s=15.0):
         if time.perf_counter() - t_start > 2 * budget_s:
             break
     us_per_call = t_full / n * 1e6 / CALLS_PER_STEP
+    wall = time.perf_counter() - t_start
+    # the same step on one BLAS thread, on a bounded share of every call's
+    # output channels (about 5 s), scaled to the full step
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"):
+            probe = time_oracle_step(ow, 1.0 / 64)
+            frac = min(1.0, max(1.0 / 64, 5.0 / max(probe, 1e-9)))
+            single = round(time_oracle_step(ow, frac) * 1e6 / CALLS_PER_STEP, 1)
+    except ImportError:
+        pass
     return {"value": round(us_per_call, 1), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{n} full oracle steps (6 calls each: dequantize-exact + fp64 GEMM, "
-                      f"storage packed beforehand), {time.perf_counter() - t_start:.1f} s"}
+                      f"storage packed beforehand), {wall:.1f} s",
+            "single_core_value": single,
+            "quantize_pack_s": {f: round(v, 3) for f, v in ow.pack_s.items()}}
 
 
 def run_reference(args, rank, world):
