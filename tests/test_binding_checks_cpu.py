@@ -77,3 +77,27 @@ def test_require_checks_in_order():
         _require(good, "x", nbytes=1024)
     with pytest.raises(ValueError, match="expected"):
         _require(good, "x", device=torch.device("cuda", 1))
+
+
+def test_layer_cannot_be_copied_or_pickled():
+    import copy
+    import pickle
+
+    lin = _layer()
+    for fn in (copy.copy, copy.deepcopy, pickle.dumps):
+        with pytest.raises(TypeError, match="handle"):
+            fn(lin)
+
+
+def test_dqlinear_module_cannot_be_deep_copied():
+    # nn.Module deepcopy reaches the layer and stops there, instead of
+    # producing two owners of one handle
+    import copy
+
+    from weight_only_quantized_prologue_b200 import module as M
+
+    mod = M.DQLinear.__new__(M.DQLinear)
+    torch.nn.Module.__init__(mod)
+    mod.layer = _layer()
+    with pytest.raises(TypeError, match="handle"):
+        copy.deepcopy(mod)

@@ -193,6 +193,17 @@ class QuantizedLinear:
     def handle(self):
         return self._h
 
+    # the object owns a library handle (device memory freed by close), so a
+    # copy would destroy it twice and a pickle would carry a dead pointer
+    def __copy__(self):
+        raise TypeError("QuantizedLinear owns a device handle and cannot be copied; build another layer")
+
+    def __deepcopy__(self, memo):
+        self.__copy__()
+
+    def __reduce__(self):
+        raise TypeError("QuantizedLinear owns a device handle and cannot be pickled")
+
     def close(self):
         if self._h is not None:
             dqgemm_destroy(self._h)
