@@ -31,6 +31,14 @@
  *     synchronous.  Nothing aborts, throws or traps across this boundary.
  *   - Device pointers must be 16-byte aligned (DQ_ERR_ALIGNMENT otherwise).
  *   - The library never frees or retains caller memory.
+ *   - A handle belongs to the device that was current at dqgemm_create.  Every
+ *     later call on it must be made with that device current, with x, y and
+ *     the stream on that device (not checked: the launch goes to the current
+ *     device).
+ *   - The run entry points keep no host state between calls, so one handle
+ *     may be run from several host threads and streams at once.
+ *     dqgemm_destroy must not overlap any other call on the same handle, nor
+ *     any of its kernels still in flight.
  */
 #ifndef DQGEMM_H
 #define DQGEMM_H

@@ -11,6 +11,7 @@ def _layer(fmt="int4", K=256, N=128):
     # a layer object without a library handle: only the argument checks run
     lin = dq.QuantizedLinear.__new__(dq.QuantizedLinear)
     lin._h, lin.fmt, lin.K, lin.N, lin.act_scale = None, fmt, K, N, None
+    lin.device, lin._check_current = torch.device("cuda", 0), False
     return lin
 
 
@@ -101,3 +102,24 @@ def test_dqlinear_module_cannot_be_deep_copied():
     mod.layer = _layer()
     with pytest.raises(TypeError, match="handle"):
         copy.deepcopy(mod)
+
+
+def test_x_on_another_device_is_rejected():
+    # the handle belongs to cuda:0; an operand on cuda:1 would be read through
+    # a pointer of the wrong device
+    from weight_only_quantized_prologue_b200 import _fits
+
+    class OnDevice1:
+        dtype, is_cuda, shape = torch.bfloat16, True, (4, 256)
+        device = torch.device("cuda", 1)
+
+        def dim(self):
+            return 2
+
+        def is_contiguous(self):
+            return True
+
+    lin = _layer()
+    assert not _fits(OnDevice1(), 256, torch.bfloat16, device=lin.device)
+    with pytest.raises(ValueError, match="expected cuda:0"):
+        lin(OnDevice1())

@@ -90,6 +90,9 @@ class QuantizedLinear:
         if bias is not None:
             _require(bias, "bias", shape=(N,), dtype=torch.bfloat16, device=packed.device)
         self.fmt, self.K, self.N = fmt, K, N
+        self.device = packed.device               # the handle belongs to this device
+        # with one visible GPU the current device can only be this one
+        self._check_current = torch.cuda.device_count() > 1
         self.act_scale = float(global_scale) if fmt == "fp8_static" else None
         self._h = dqgemm_create(fmt, K, N, packed, scales, global_scale, bias)
 
@@ -113,10 +116,16 @@ class QuantizedLinear:
         return cls(fmt, K, N, packed, scales, g, bias)
 
     def _check_x(self, x, dtype, name="x"):
-        if not _fits(x, self.K, dtype):
+        if not _fits(x, self.K, dtype, device=self.device):
             if getattr(x, "dim", lambda: 0)() != 2:
                 raise ValueError(f"{name} must be 2-D [M, {self.K}]")
-            _require(x, name, shape=(x.shape[0], self.K), dtype=dtype)
+            _require(x, name, shape=(x.shape[0], self.K), dtype=dtype, device=self.device)
+        if self._check_current:
+            import torch
+
+            if torch.cuda.current_device() != self.device.index:
+                raise ValueError(f"the layer lives on {self.device}; make it the current device "
+                                 f"(torch.cuda.set_device / torch.cuda.device) before calling it")
         return x.shape[0]
 
     def _out(self, out, M, dtype, device):
@@ -179,7 +188,7 @@ class QuantizedLinear:
     def dequantize(self, stream=None):
         import torch
 
-        w = torch.empty((self.N, self.K), dtype=torch.bfloat16, device="cuda")
+        w = torch.empty((self.N, self.K), dtype=torch.bfloat16, device=self.device)
         dqgemm_dequantize(self._h, w, stream)
         return w
 
