@@ -169,7 +169,9 @@ dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x,
  *   FP8    s[n] = max|W[n,:]|/448; c = e4m3(W/s[n]) (0 for a zero row)
  *   INT4 asymmetric  lo = min(0, min W), hi = max(0, max W) per group;
  *          s = bf16(f32(hi - lo)/15); z = clamp(rne(-lo/s), 0, 15);
- *          c = clamp(rne(W/s) + z, 0, 15); s == 0 -> c = 0, z = 0
+ *          c = clamp(rne(W/s) + z, 0, 15); s == 0 -> c = 0, z = 0; a group
+ *          whose range hi - lo exceeds the fp32 maximum (weights of both
+ *          signs near +-3.4e38) gets an infinite scale: it is not rejected
  * `global_scale` (host, may be NULL) receives g for NVFP4 and 1 otherwise.
  * DQ_ERR_INVALID_ARG if W holds a non-finite value. */
 dqgemm_status dqgemm_pack_host(dqgemm_format fmt, const float* W, int K, int N,
