@@ -39,6 +39,16 @@
  *     may be run from several host threads and streams at once.
  *     dqgemm_destroy must not overlap any other call on the same handle, nor
  *     any of its kernels still in flight.
+ *
+ * Environment variables, each read once per process, for tuning and tests
+ * only (results do not depend on them except through the split, which only
+ * changes the fp32 summation order):
+ *   DQGEMM_TIMEOUT_MS   limit of every device-side wait (default 2000 ms).
+ *   DQGEMM_PDL=0        launch without programmatic dependent launch.
+ *   DQGEMM_SPLIT=S      force the split-K depth to the largest power of two
+ *                       <= min(S, 8, K/128) that fits the cluster limits.
+ *   DQGEMM_CTAS_PER_SM  2 lets the split plan count two resident CTAs per SM
+ *                       for the skinny tiles (default 1).
  */
 #ifndef DQGEMM_H
 #define DQGEMM_H
