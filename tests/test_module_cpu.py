@@ -26,3 +26,18 @@ def test_calibration_records_the_input_range_of_every_linear():
     assert scales["2"] == float(torch.tensor(a2, dtype=torch.float32) / 448.0)
     # hooks are removed afterwards
     assert not model[0]._forward_pre_hooks and not model[2]._forward_pre_hooks
+
+
+def test_op_traces_through_torch_export():
+    # the pages' flow starts from torch.export; a model calling the op exports
+    # with the op as one node, shaped by the fake implementation alone (no
+    # library call, so no GPU)
+    class Wrap(torch.nn.Module):
+        def forward(self, x):
+            return torch.relu(torch.ops.dqgemm.linear(x, 12345, 64))
+
+    ep = torch.export.export(Wrap(), (torch.empty(4, 128, dtype=torch.bfloat16),))
+    targets = [n.target for n in ep.graph.nodes if n.op == "call_function"]
+    assert torch.ops.dqgemm.linear.default in targets
+    out = [n for n in ep.graph.nodes if n.op == "output"][0].args[0][0]
+    assert tuple(out.meta["val"].shape) == (4, 64) and out.meta["val"].dtype == torch.bfloat16
