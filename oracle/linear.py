@@ -179,9 +179,12 @@ def calibrate_static_mlp(batches, w1, w2):
     Q/DQ").  Observers watch the float (bf16) model: layer 1's input is the
     batch itself, layer 2's input is h = bf16(x . w1^T).
     Reading: the float model's Linear is taken as the exact product rounded
-    once to bf16.  Returns (s_x1, s_x2).  Parity unpinned (the pages print no
-    scale values); both the oracle and the GPU path receive these scales as
-    inputs, so GEMM parity does not depend on them."""
+    once to bf16.  Returns (s_x1, s_x2).  The pages print no scale values;
+    parity is pinned by invariants (batch order, monotonicity under an extra
+    batch, exact 2^j equivariance) and by constructed cases that fix the
+    symmetric range and the bf16 rounding of layer 1's output.  Both the
+    oracle and the GPU path receive these scales as inputs, so GEMM parity
+    does not depend on them."""
     lo1 = hi1 = lo2 = hi2 = None
     for x in batches:
         x = np.asarray(x, dtype=np.float64)

@@ -97,3 +97,29 @@ def test_sqnr_limits():
     a = np.array([3.0, 4.0])
     assert np.isclose(L.sqnr(a, a), 20 * np.log10(5.0 / 1e-12))
     assert np.isclose(L.sqnr(a, np.zeros(2)), 0.0)
+
+
+def test_calibration_invariants():
+    # order of the batches does not matter, an extra batch never lowers a
+    # scale, and scaling every batch by 2^j scales both scales by exactly 2^j
+    rng = np.random.default_rng(5)
+    w1 = rng.uniform(-0.1, 0.1, (16, 8))
+    w2 = rng.uniform(-0.1, 0.1, (4, 16))
+    batches = [F.bf16(rng.standard_normal((3, 8)) * (1 + i)) for i in range(5)]
+    s = L.calibrate_static_mlp(batches, w1, w2)
+    assert L.calibrate_static_mlp(batches[::-1], w1, w2) == s
+    s4 = L.calibrate_static_mlp(batches[:4], w1, w2)
+    assert s4[0] <= s[0] and s4[1] <= s[1]
+    for j in (-4, 3):
+        sj = L.calibrate_static_mlp([b * 2.0 ** j for b in batches], w1, w2)
+        assert sj == (s[0] * 2.0 ** j, s[1] * 2.0 ** j)
+
+
+def test_calibration_layer2_sees_bf16_output_and_negative_side():
+    # layer 1's output is observed after rounding to bf16: 1 + 2^-10 is not a
+    # bf16 value and rounds to 1; the negative side dominates the range here
+    x = np.array([[1.0, 0.0], [0.0, -5.0]])
+    w1 = np.array([[1.0 + 2.0 ** -10, 0.0]])
+    s1, s2 = L.calibrate_static_mlp([x], w1, np.eye(1))
+    assert s1 == float(F.f32(5.0 / 448))
+    assert s2 == float(F.f32(1.0 / 448))
