@@ -207,8 +207,9 @@ def static_mlp(x, s_x1, q_w1, s_w1, s_x2, q_w2, s_w2):
 def sqnr(a, b):
     """Signal-to-quantization-noise ratio in dB, 20 log10(|a| / |a - b|) with
     the noise norm clamped at 1e-12 (the helper on the static FP8 page,
-    "Imports" section).  Diagnostic only: the pages print no values, so it
-    is parity unpinned."""
+    "Imports" section).  Diagnostic only: the pages print no SQNR values to
+    compare against; the function itself is pinned by closed forms (b = a
+    gives the clamp, b = 0 gives 0 dB, b = a (1 + eps) gives -20 log10 eps)."""
     a = np.asarray(a, dtype=np.float64).ravel()
     b = np.asarray(b, dtype=np.float64).ravel()
     noise = max(np.linalg.norm(a - b), 1e-12)

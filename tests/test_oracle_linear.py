@@ -123,3 +123,10 @@ def test_calibration_layer2_sees_bf16_output_and_negative_side():
     s1, s2 = L.calibrate_static_mlp([x], w1, np.eye(1))
     assert s1 == float(F.f32(5.0 / 448))
     assert s2 == float(F.f32(1.0 / 448))
+
+
+def test_sqnr_closed_form():
+    # b = a (1 + eps) gives |a| / |a - b| = 1 / eps exactly: 20 log10(1 / eps) dB
+    a = np.random.default_rng(9).standard_normal(1000)
+    for k in (3, 10, 20):
+        assert np.isclose(L.sqnr(a, a * (1 + 2.0 ** -k)), 20 * k * np.log10(2.0), rtol=1e-9)
