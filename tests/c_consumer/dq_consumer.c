@@ -81,12 +81,14 @@ static int do_pack(int fmt, int K, int N, const char* win, const char* out) {
 }
 
 static int do_errors(void) {
-  float w[256];
-  uint8_t packed[256], scales[16];
+  /* malloc returns memory aligned for any type: 16 bytes on x86-64 */
+  float* w = (float*)calloc(256, sizeof(float));
+  uint8_t* packed = (uint8_t*)calloc(256, 1);
+  uint8_t* scales = (uint8_t*)calloc(16, 1);
   float g;
   dqgemm_handle h = NULL;
   dqgemm_plan plan;
-  memset(w, 0, sizeof w);
+  if (!w || !packed || !scales) return 2;
   printf("pack_null_weight %d\n", (int)dqgemm_pack_host(DQ_INT4_G128, NULL, 128, 2, packed, scales, &g));
   printf("pack_k_not_group %d\n", (int)dqgemm_pack_host(DQ_INT4_G128, w, 100, 2, packed, scales, &g));
   printf("pack_unknown_format %d\n", (int)dqgemm_pack_host((dqgemm_format)9, w, 128, 2, packed, scales, &g));
@@ -99,7 +101,19 @@ static int do_errors(void) {
   printf("plan_null_handle %d\n", (int)dqgemm_get_plan(NULL, 1, &plan));
   printf("destroy_null %d\n", (int)dqgemm_destroy(NULL));
   printf("last_error_null %d\n", (int)dqgemm_last_error(NULL));
+  /* 16-byte alignment is checked before any device access */
+  printf("create_misaligned %d\n",
+         (int)dqgemm_create(&h, DQ_INT4_G128, 128, 128, packed + 1, scales, 1.f, NULL));
+  printf("pack_device_misaligned %d\n",
+         (int)dqgemm_pack_device(DQ_INT4_G128, w + 1, 128, 2, packed, scales, NULL, NULL));
+  printf("pack_device_null %d\n", (int)dqgemm_pack_device(DQ_INT4_G128, NULL, 128, 2, packed, scales, NULL, NULL));
+  printf("act_quant_m0 %d\n", (int)dqgemm_quantize_act_fp8(packed, 0, 16, 1.f, packed, NULL));
+  printf("act_quant_zero_scale %d\n", (int)dqgemm_quantize_act_fp8(packed, 1, 16, 0.f, packed, NULL));
+  printf("act_quant_nan_scale %d\n", (int)dqgemm_quantize_act_fp8(packed, 1, 16, NAN, packed, NULL));
   printf("status_string %s\n", dqgemm_status_string(DQ_ERR_INVALID_ARG));
+  free(w);
+  free(packed);
+  free(scales);
   return 0;
 }
 

@@ -91,6 +91,10 @@ def test_c_argument_errors(consumer):
                  "last_error_null"):
         assert got[case] == invalid, (case, got[case])
     assert got["create_null_weight"] == f"{invalid} 1"       # and *out was set to NULL
+    align = str(dq._native.DQ_ERR_ALIGNMENT)
+    assert got["create_misaligned"] == align and got["pack_device_misaligned"] == align
+    for case in ("pack_device_null", "act_quant_m0", "act_quant_zero_scale", "act_quant_nan_scale"):
+        assert got[case] == invalid, (case, got[case])
     assert got["status_string"] == dq.dqgemm_status_string(dq._native.DQ_ERR_INVALID_ARG)
 
 
