@@ -29,7 +29,8 @@
  *     stream).  Calls that take a stream are asynchronous on it.
  *   - Every entry point returns a dqgemm_status.  Argument checks are
  *     synchronous.  Nothing aborts, throws or traps across this boundary.
- *   - Device pointers must be 16-byte aligned (DQ_ERR_ALIGNMENT otherwise).
+ *   - Device pointers must be 16-byte aligned (DQ_ERR_ALIGNMENT otherwise),
+ *     except where an entry point says so.
  *   - The library never frees or retains caller memory.
  *   - A handle belongs to the device that was current at dqgemm_create.  Every
  *     later call on it must be made with that device current, with x, y and
@@ -164,7 +165,9 @@ dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream);
 /* Static-FP8 activation quantization (the Q node of the static FP8 page's
  * "Graph after export"): q[m,k] = e4m3(f32(x[m,k] / s_x)), IEEE division,
  * round to nearest even, saturating to +-448.  x: device bf16 [M, K];
- * q: device u8 [M, K]; s_x > 0. */
+ * q: device u8 [M, K]; s_x finite and > 0, M >= 1, K >= 1, else
+ * DQ_ERR_INVALID_ARG.  Element-wise, so x and q need only their natural
+ * alignment (the one exception to the 16-byte rule above). */
 dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x,
                                       void* q, void* stream);
 
