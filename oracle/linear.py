@@ -198,7 +198,10 @@ def calibrate_static_mlp(batches, w1, w2):
 
 def static_mlp(x, s_x1, q_w1, s_w1, s_x2, q_w2, s_w2):
     """The page's two-layer model after static FP8 Q/DQ: h = bf16(layer1),
-    y = bf16(layer2(Q(h))).  Returns (h, y) as fp64 values of bf16."""
+    y = bf16(layer2(Q(h))).  Returns (h, y) as fp64 values of bf16.
+    Parity: pinned by a two-layer case worked by hand in which the bf16
+    rounding of h, layer 2's own activation scale, its Q node and the
+    orientation of W1 each change the result."""
     h = bf16(static_linear(quantize_act_fp8(x, s_x1), s_x1, q_w1, s_w1))
     y = bf16(static_linear(quantize_act_fp8(h, s_x2), s_x2, q_w2, s_w2))
     return h, y

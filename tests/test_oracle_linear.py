@@ -130,3 +130,28 @@ def test_sqnr_closed_form():
     a = np.random.default_rng(9).standard_normal(1000)
     for k in (3, 10, 20):
         assert np.isclose(L.sqnr(a, a * (1 + 2.0 ** -k)), 20 * k * np.log10(2.0), rtol=1e-9)
+
+
+def test_static_mlp_hand_worked_two_layers():
+    """The static page's two-layer model after Q/DQ, worked by hand on a
+    1 x 2 -> 2 -> 1 case whose numbers force every step to matter.
+      layer 1: s_x1 = 1/16, x = [1/8, -3/8]  -> codes [2, -6]
+               W1 codes [[1, 1/2], [-2, 1]]  -> sums [2 - 3, -4 - 6] = [-1, -10]
+               s_w1 = [f32(545.6), 128]      -> h = bf16([-34.0999985, -80]) = [-34, -80]
+      layer 2: s_x2 = 1/4  -> h / s_x2 = [-136, -320]; -136 lies halfway
+               between the e4m3 points 128 and 144 and rounds to the even
+               mantissa, 128, so the codes are [-128, -320]
+               W2 codes [[3, -3/2]], s_w2 = [2] -> sum 96 -> y = 96 * 1/4 * 2 = 48
+    Each plausible slip gives another y: without the bf16 rounding of h,
+    -34.0999985 / (1/4) rounds to -144 and y = 24; with layer 1's scale in
+    layer 2, h / (1/16) saturates at -448 twice and y = -84; without the
+    layer-2 Q node y = 36; with W1 transposed the layer-1 sums are [14, -5]."""
+    e4m3 = {1.0: 0x38, 0.5: 0x30, -2.0: 0xC0, 3.0: 0x44, -1.5: 0xBC}   # OCP E4M3 bit patterns
+    q_w1 = np.array([[e4m3[1.0], e4m3[0.5]], [e4m3[-2.0], e4m3[1.0]]], dtype=np.uint8)
+    q_w2 = np.array([[e4m3[3.0], e4m3[-1.5]]], dtype=np.uint8)
+    s_w1 = np.array([545.6, 128.0], dtype=np.float32)
+    s_w2 = np.array([2.0], dtype=np.float32)
+    x = np.array([[0.125, -0.375]])
+    h, y = L.static_mlp(x, 0.0625, q_w1, s_w1, 0.25, q_w2, s_w2)
+    assert h.tolist() == [[-34.0, -80.0]]
+    assert y.tolist() == [[48.0]]
