@@ -110,7 +110,14 @@ typedef struct dqgemm_s* dqgemm_handle;
  * memory owned by the handle (the analogue of the INT4 page's "re-packs ...
  * into an INT4 constant at build time", "Export and compile").  The caller may
  * free its buffers afterwards; the weights are immutable for the handle's
- * life.  Synchronizes the device.  On error *out is set to NULL. */
+ * life.  Synchronizes the device.  On error *out is set to NULL.
+ * Stored codes outside what the formats define are refused with
+ * DQ_ERR_INVALID_ARG: a NaN weight code (0x7F / 0xFF) of the FP8 formats, an
+ * NVFP4 block scale that is negative or NaN (the block scales are
+ * non-negative E4M3), an MXFP4 exponent 0xFF.  An MXFP4 handle whose largest
+ * block exponent code emax exceeds 128 needs every block holding a nonzero
+ * element to have a code >= emax - 133 (the bf16 operand of the prologue
+ * covers a span of 2^133 exactly); DQ_ERR_UNSUPPORTED otherwise. */
 dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt, int K, int N,
                             const void* packed_w, const void* scales,
                             float global_scale, const void* bias);
@@ -207,10 +214,12 @@ dqgemm_status dqgemm_pack_device(dqgemm_format fmt, const float* W, int K, int N
  * amax: its two-pass reduction keeps up to 4096 partial maxima (one per
  * 65536 weights) in a static device array that every GPU loading the library
  * holds (16 KB) until exit, so NVFP4 requires N*K <= 4096*65536 and returns
- * DQ_ERR_UNSUPPORTED beyond that; the other formats need no scratch.  The
- * first call on a device looks up the array's device address (do it before
- * any stream capture).  All calls share the array: calls whose kernels
- * overlap on the GPU race with each other.  If `global_scale` (host) is not
+ * DQ_ERR_UNSUPPORTED beyond that; the other formats need no scratch.  Each
+ * NVFP4 call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress); the first such call on a device may load the
+ * library's device code, so make it before any stream capture.  All calls
+ * share the array: calls whose kernels overlap on the GPU race with each
+ * other.  If `global_scale` (host) is not
  * NULL the call synchronizes `stream` and stores g there. */
 dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt, const float* W, int K, int N,
                                          void* packed, void* scales, float* global_scale,

@@ -13,13 +13,19 @@ def pytest_configure(config):
 
 
 def pytest_sessionstart(session):
-    # a fresh checkout has no libdqgemm.so (built files are not versioned):
-    # build it once, in-tree, so the ABI tests have a library to load (nvcc
-    # cross-compiles for sm_100a without a GPU)
+    # build (or rebuild after a source edit) libdqgemm.so in-tree so the tests
+    # load the library of the sources they test; build() returns at once when
+    # the library is newer than every source.  nvcc cross-compiles for sm_100a
+    # without a GPU; without nvcc the oracle-only tests still run.
+    import shutil
+    import warnings
+
     from weight_only_quantized_prologue_b200 import build
 
-    if not os.path.exists(build.LIB):
-        build.build()
+    if shutil.which(build.nvcc()) is None and not os.path.exists(build.nvcc()):
+        warnings.warn("nvcc not found: libdqgemm.so is not (re)built; the ABI tests use whatever library exists")
+        return
+    build.build()
 
 
 @pytest.fixture(scope="session")

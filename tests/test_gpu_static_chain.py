@@ -35,6 +35,16 @@ def test_quantized_out_equals_run_then_quantize(fmt, M, N):
         torch.cuda.synchronize()
         assert lin.last_error() == 0
         assert torch.equal(q, q_ref)
+        # against the oracle: y within tolerance of the fp64 reference (the GPU
+        # packer's storage equals the oracle's byte for byte), and the codes
+        # exactly the oracle's Q node applied to that bf16 y
+        st = L.quantize_pack("fp8" if fmt == "fp8_static" else fmt, W.numpy().astype(np.float64))
+        wdq = L.dequant_exact("fp8" if fmt == "fp8_static" else fmt, st["packed"], st["scales"], st["global_scale"])
+        xv = bf16_values(x)
+        x_eff = static_effective_x(xv, s_in) if fmt == "fp8_static" else xv
+        yv = bf16_values(y)
+        check_close(yv, L.linear_ref(x_eff, wdq, None if fmt == "fp8_static" else bf16_values(b)), x_eff, wdq)
+        assert np.array_equal(q.cpu().numpy(), L.quantize_act_fp8(yv, s_out))
     finally:
         lin.close()
 
@@ -50,10 +60,26 @@ def test_two_layer_static_mlp_chained_through_codes(M):
     l2 = dq.QuantizedLinear.from_float("fp8_static", w2.float().cuda(), None, act_scale=s2)
     try:
         x = synthetic.activations(M, 256, seed=9).cuda()
-        y_plain = l2(l1(x))
-        y_chain = l2.from_codes(l1.quantized_out(x, s2))
+        h = l1(x)
+        y_plain = l2(h)
+        q = l1.quantized_out(x, s2)
+        y_chain = l2.from_codes(q)
         torch.cuda.synchronize()
         assert torch.equal(y_chain.view(torch.int16), y_plain.view(torch.int16))
+        # against the oracle: layer 1 within tolerance, the chained codes
+        # exactly the oracle's Q node on the GPU's h, and layer 2 on those
+        # codes within tolerance
+        st1 = L.quantize_pack("fp8", w1.float().numpy().astype(np.float64))
+        st2 = L.quantize_pack("fp8", w2.float().numpy().astype(np.float64))
+        wdq1 = L.dequant_exact("fp8", st1["packed"], st1["scales"])
+        wdq2 = L.dequant_exact("fp8", st2["packed"], st2["scales"])
+        xv, hv = bf16_values(x), bf16_values(h)
+        x1 = static_effective_x(xv, s1)
+        check_close(hv, L.linear_ref(x1, wdq1), x1, wdq1)
+        q_ref = L.quantize_act_fp8(hv, s2)
+        assert np.array_equal(q.cpu().numpy(), q_ref)
+        x2 = static_effective_x(hv, s2)
+        check_close(bf16_values(y_chain), L.static_linear(q_ref, s2, st2["packed"], st2["scales"]), x2, wdq2)
     finally:
         l1.close()
         l2.close()

@@ -59,3 +59,21 @@ def test_noalloc_packer_rejects_tensors_beyond_its_scratch():
     st = dq._native.lib().dqgemm_pack_device_noalloc(dq.FORMATS["nvfp4"], W.data_ptr(), 16400, 16384,
                                                      out.data_ptr(), out.data_ptr(), None, None)
     assert st == dq._native.DQ_ERR_UNSUPPORTED
+
+
+def test_noalloc_nvfp4_many_partials_with_the_maximum_in_the_last_partial_chunk():
+    # 1040 x 16400 weights: 261 partial maxima (more than one per thread of the
+    # final reduction's 256) and a last chunk holding only 16640 weights; the
+    # tensor maximum sits in that last, partial chunk.  The second call is
+    # smaller and its maximum is in its first chunk, so a stale partial left
+    # by the first call would raise its global scale.
+    for call, (N, K, where) in enumerate([(1040, 16400, -1), (512, 2048, 0)]):
+        W = _weights(N, K, seed=20 + call, scale=0.5)
+        flat = W.view(-1)
+        flat[where] = 40.0 if call == 0 else 7.0
+        ref = _pack(dq.dqgemm_pack_device, "nvfp4", W)
+        got = _pack(dq.dqgemm_pack_device_noalloc, "nvfp4", W)
+        assert np.array_equal(got[0], ref[0]), f"call {call}: packed codes differ"
+        assert np.array_equal(got[1], ref[1]), f"call {call}: scales differ"
+        assert np.float32(got[2]) == np.float32(ref[2]), f"call {call}: global scale differs"
+        assert np.float32(got[2]) == np.float32(np.float32(40.0 if call == 0 else 7.0) / np.float32(2688.0))

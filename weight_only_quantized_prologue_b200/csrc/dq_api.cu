@@ -6,7 +6,6 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
-#include <mutex>
 #include <vector>
 
 #include "dq_aux.cuh"
@@ -409,6 +408,43 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
 
 dqgemm_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA; }
 
+// Codes the canonical storage may hold (the packers produce nothing else):
+//   FP8 formats  no NaN weight code (0x7F / 0xFF)
+//   NVFP4        block scales are non-negative finite E4M3 (no sign bit, no 0x7F)
+//   MXFP4        no NaN exponent (0xFF); and, because the prologue's bf16
+//                operand e2m1 * 2^(e - 127 - J) (J = max(0, emax - 128),
+//                undone in the epilogue) must not fall below the smallest
+//                bf16 subnormal, every block with a nonzero element has an
+//                exponent code >= emax - 133 when emax > 128
+//                (DQ_ERR_UNSUPPORTED otherwise: the span of 2^133 between a
+//                handle's block scales is past what it represents exactly)
+dqgemm_status check_codes(int fmt, int K, int N, const std::vector<uint8_t>& hp, const std::vector<uint8_t>& hs) {
+  if (fmt == FMT_FP8 || fmt == FMT_FP8S) {
+    for (uint8_t c : hp)
+      if ((c & 0x7F) == 0x7F) return DQ_ERR_INVALID_ARG;
+  } else if (fmt == FMT_NVFP4) {
+    for (uint8_t c : hs)
+      if (c >= 0x7F) return DQ_ERR_INVALID_ARG;
+  } else if (fmt == FMT_MXFP4) {
+    int cmax = 0;
+    for (uint8_t c : hs) {
+      if (c == 255) return DQ_ERR_INVALID_ARG;
+      cmax = std::max<int>(cmax, c);
+    }
+    if (cmax > 128) {
+      const int blocks = K / 32;
+      for (int n = 0; n < N; ++n)
+        for (int b = 0; b < blocks; ++b) {
+          if (hs[(size_t)n * blocks + b] >= cmax - 133) continue;
+          const uint8_t* e = &hp[(size_t)n * (K / 2) + (size_t)b * 16];
+          for (int i = 0; i < 16; ++i)
+            if (e[i] & 0x77) return DQ_ERR_UNSUPPORTED;   // a nonzero magnitude in either nibble
+        }
+    }
+  }
+  return DQ_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -458,6 +494,8 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   if (cudaMemcpy(hp.data(), packed_w, hp.size(), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(hs.data(), scales, hs.size(), cudaMemcpyDeviceToHost) != cudaSuccess)
     return DQ_ERR_CUDA;
+  st = check_codes(fmt, K, N, hp, hs);
+  if (st != DQ_OK) return st;
 
   dqgemm_s* h = new dqgemm_s();
   h->fmt = fmt;
@@ -475,7 +513,6 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   } else if (fmt == FMT_MXFP4) {
     int cmax = 0;
     for (uint8_t c : hs) cmax = std::max<int>(cmax, c);
-    if (cmax == 255) { delete h; return DQ_ERR_INVALID_ARG; }   // NaN scale
     const int J = std::max(0, cmax - 128);
     h->mx_bias = 126 - J;
     h->sigma = std::ldexp(1.f, J);
@@ -709,29 +746,19 @@ constexpr long long kNoAllocChunk = 65536;         // weights reduced per partia
 // [0, 4096): partial maxima; [4096]: amax bits; [4097]: global scale g
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxPartials + 2];
 
-constexpr int kMaxDevices = 64;
-float* g_noalloc_ptr[kMaxDevices] = {};
-std::mutex g_noalloc_mu;
-
-// Device address of the scratch on the current device, looked up once per
-// device (the symbol's host-side name is not a device address).
+// Device address of the scratch on the current device.  The symbol's
+// host-side name is not a device address, so it is looked up on every call:
+// a cached address would go stale if the device's primary context were torn
+// down and the library's device code loaded again.
 float* noalloc_scratch(dqgemm_status* st) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
     *st = DQ_ERR_CUDA;
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-      *st = DQ_ERR_CUDA;
-      return nullptr;
-    }
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
-  }
   *st = DQ_OK;
-  return g_noalloc_ptr[dev];
+  return static_cast<float*>(p);
 }
 }  // namespace
 
