@@ -160,7 +160,9 @@ dqgemm_status dqgemm_run_quantized_out(dqgemm_handle h, const void* x, int M, vo
 dqgemm_status dqgemm_run_fp8_static_quantized_out(dqgemm_handle h, const void* q, int M, void* q_out,
                                                   float s_out, void* stream);
 
-/* Release the handle and its device memory (synchronizes the device). */
+/* Release the handle and its device memory.  Synchronizes the device (the
+ * CUDA runtime's cudaFree does so in any case); no kernel of the handle may
+ * still be queued or running. */
 dqgemm_status dqgemm_destroy(dqgemm_handle h);
 
 /* Debug: write the dequantized weight as bf16 [N, K] (device) from the
@@ -225,9 +227,24 @@ dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt, const float* W, int 
                                          void* packed, void* scales, float* global_scale,
                                          void* stream);
 
-/* Status of the last device-side check of the handle's kernels (DQ_OK or
- * DQ_ERR_TIMEOUT), then clears it.  Synchronizes the device. */
+/* Status of the device-side checks of the handle's completed kernels (DQ_OK,
+ * or DQ_ERR_TIMEOUT if a bounded wait of any of them gave up), then clears
+ * it.  The status word is host memory the kernels write into: this call does
+ * not synchronize anything, so synchronize the streams the handle's kernels
+ * ran on first (a kernel still running may report later). */
 dqgemm_status dqgemm_last_error(dqgemm_handle h);
+
+/* Test and diagnostic use: the limit, in nanoseconds, of the device-side
+ * waits of this handle's GEMM pipeline (0 restores the default, which is
+ * DQGEMM_TIMEOUT_MS or 2 s).  A wait that does not complete at once gives up
+ * when its limit has passed: the kernel then records DQ_ERR_TIMEOUT (read by
+ * dqgemm_last_error) and writes no output of the tiles it gave up on.  The
+ * waits for a CTA's own copies, tensor-core operations and received split-K
+ * partials keep a limit of at least the default, so that no kernel leaves
+ * memory that is still being written.  Calls already launched keep the limit
+ * they were launched with.  DQ_ERR_INVALID_ARG for a null handle or a
+ * negative limit. */
+dqgemm_status dqgemm_set_wait_limit(dqgemm_handle h, long long timeout_ns);
 
 /* Diagnostic: launch a kernel whose only wait can never complete and which
  * must give up after `timeout_us` microseconds; returns DQ_ERR_TIMEOUT when
@@ -247,6 +264,8 @@ typedef struct {
   int smem_bytes;       /* dynamic shared memory per CTA */
   long long workspace_bytes; /* global split-K scratch the plan needs (0: partials stay on chip) */
   long long weight_bytes;    /* packed weight + scale bytes streamed per call */
+  int x_stages;         /* activation-tile ring depth (128-k stages) */
+  int max_cta_stages;   /* most 128-k weight stages one CTA streams */
 } dqgemm_plan;
 
 dqgemm_status dqgemm_get_plan(dqgemm_handle h, int M, dqgemm_plan* plan);

@@ -87,9 +87,10 @@ def test_two_layer_static_mlp_chained_through_codes(M):
 
 @pytest.mark.parametrize("fmt", ["int4", "nvfp4", "fp8_static", "int4_asym"])
 def test_persistent_whole_tile_path_matches_oracle(fmt):
-    # 2 x 80 output tiles of 128 x 128 > the SM count: no split-K, each CTA
-    # loops over whole tiles
-    M, K, N = 256, 256, 10240
+    # more output tiles than SMs with either x tile (2 x 160 tiles of 128
+    # rows, or 160 tiles of 256 rows): no split-K, each CTA loops over
+    # whole tiles
+    M, K, N = 256, 256, 20480
     x, W, b = synthetic.linear_inputs(M, K, N, seed=21)
     W = W.numpy().astype(np.float64)
     xv = bf16_values(x)

@@ -1,0 +1,61 @@
+"""The GEMM's own bounded-wait path, run on the GPU without a fault.
+
+A handle's pipeline waits get a limit so short that the first wait which
+does not complete at once gives up (dqgemm_set_wait_limit, a test and
+diagnostic knob; the shared default is not touched).  Every CTA then takes
+its abort path: it drains its own copies and tensor-core operations, still
+sends its (invalid) split-K partials so that every receive of the cluster
+completes, and writes no output.  The call must report DQ_ERR_TIMEOUT,
+leave y untouched, and leave the context usable: the same handle with the
+default limit restored, and the next call, give the oracle's result."""
+
+import numpy as np
+import pytest
+import torch
+
+import weight_only_quantized_prologue_b200 as dq
+from oracle import linear as L
+from weight_only_quantized_prologue_b200 import synthetic
+
+from gpu_util import bf16_values, check_close, make_layer, static_effective_x
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "fp8", "fp8_static"])
+@pytest.mark.parametrize("M,K,N", [(32, 3072, 4096), (1, 1024, 512), (256, 256, 19200)])
+def test_gemm_wait_limit_expires_then_context_recovers(fmt, M, K, N):
+    x, w, b = synthetic.linear_inputs(M, K, N, seed=31)
+    W = w.numpy().astype(np.float64)
+    xv = bf16_values(x)
+    s_x = L.act_scale(xv.min(), xv.max())
+    h, st, wdq = make_layer(fmt, W, b.cuda(), act_scale=s_x)
+    try:
+        plan = dq.dqgemm_get_plan(h, M)
+        xc = x.cuda()
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dq.dqgemm_set_wait_limit(h, 1)
+        dq.dqgemm_run(h, xc, M, y)
+        torch.cuda.synchronize()
+        assert dq.dqgemm_last_error(h) == dq._native.DQ_ERR_TIMEOUT, plan
+        assert torch.isnan(y.float()).all(), "an aborted call wrote output"
+        dq.dqgemm_set_wait_limit(h, 0)          # back to the default
+        dq.dqgemm_run(h, xc, M, y)
+        torch.cuda.synchronize()
+        assert dq.dqgemm_last_error(h) == 0
+        x_eff = static_effective_x(xv, s_x) if fmt == "fp8_static" else xv
+        check_close(bf16_values(y), L.linear_ref(x_eff, wdq, bf16_values(b)), x_eff, wdq)
+    finally:
+        dq.dqgemm_destroy(h)
+
+
+def test_wait_limit_rejects_bad_arguments():
+    x, w, b = synthetic.linear_inputs(1, 256, 128, seed=3)
+    h, _, _ = make_layer("int4", w.numpy().astype(np.float64))
+    try:
+        lib = dq._native.lib()
+        assert lib.dqgemm_set_wait_limit(h, -1) == dq._native.DQ_ERR_INVALID_ARG
+        assert lib.dqgemm_set_wait_limit(None, 5) == dq._native.DQ_ERR_INVALID_ARG
+        assert lib.dqgemm_set_wait_limit(h, 0) == dq._native.DQ_OK
+    finally:
+        dq.dqgemm_destroy(h)

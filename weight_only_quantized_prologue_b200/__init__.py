@@ -28,6 +28,7 @@ from ._native import (  # noqa: F401
     dqgemm_run_fp8_static_quantized_out,
     dqgemm_run_quantized_out,
     dqgemm_selftest_timeout,
+    dqgemm_set_wait_limit,
     dqgemm_status_string,
     storage_shapes,
 )

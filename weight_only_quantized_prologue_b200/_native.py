@@ -31,7 +31,8 @@ class Plan(ctypes.Structure):
     _fields_ = [("bn", ctypes.c_int), ("m_tiles", ctypes.c_int), ("n_tiles", ctypes.c_int),
                 ("k_stages", ctypes.c_int), ("grid", ctypes.c_int), ("max_segments", ctypes.c_int),
                 ("stages", ctypes.c_int), ("smem_bytes", ctypes.c_int),
-                ("workspace_bytes", ctypes.c_longlong), ("weight_bytes", ctypes.c_longlong)]
+                ("workspace_bytes", ctypes.c_longlong), ("weight_bytes", ctypes.c_longlong),
+                ("x_stages", ctypes.c_int), ("max_cta_stages", ctypes.c_int)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -53,6 +54,7 @@ _SIGNATURES = {
     "dqgemm_last_error": [_VP],
     "dqgemm_selftest_timeout": [_I, _VP],
     "dqgemm_get_plan": [_VP, _I, ctypes.POINTER(Plan)],
+    "dqgemm_set_wait_limit": [_VP, ctypes.c_longlong],
 }
 
 _lib = None
@@ -190,6 +192,10 @@ def dqgemm_last_error(h):
 
 def dqgemm_selftest_timeout(timeout_us, stream=None):
     return lib().dqgemm_selftest_timeout(int(timeout_us), _stream(stream))
+
+
+def dqgemm_set_wait_limit(h, timeout_ns):
+    _check(lib().dqgemm_set_wait_limit(h, int(timeout_ns)), "dqgemm_set_wait_limit")
 
 
 def dqgemm_get_plan(h, M):

@@ -23,11 +23,13 @@ struct dqgemm_s {
   size_t wchunk_bytes = 0;
   float* col_scale = nullptr;       // [N] for FP8 formats
   __nv_bfloat16* bias = nullptr;    // [N] or null
-  int* status = nullptr;            // device status word
+  int* status = nullptr;            // status word as the device addresses it
+  int* status_host = nullptr;       //   ... and as the host reads it (mapped pinned memory)
   float sigma = 1.f, s_x = 1.f;
   int mx_bias = 126;
   long long weight_bytes = 0;       // canonical packed + scale bytes
   int max_clusters[4][9] = {};      // co-resident clusters per (BN index, cluster size), 0 = unknown
+  unsigned long long timeout_ns = 0;  // limit of the kernels' pipeline waits
 };
 
 namespace {
@@ -296,7 +298,22 @@ int stages_for(int bn) {
     case 16: return GemmCfg<FMT, 16>::STAGES;
     case 32: return GemmCfg<FMT, 32>::STAGES;
     case 64: return GemmCfg<FMT, 64>::STAGES;
-    default: return GemmCfg<FMT, 128>::STAGES;
+    case 128: return GemmCfg<FMT, 128>::STAGES;
+    default:
+      if constexpr (FMT == FMT_FP8S) return GemmCfg<FMT, 128>::STAGES;
+      else return GemmCfg<FMT, 256>::STAGES;
+  }
+}
+template <int FMT>
+int xstages_for(int bn) {
+  switch (bn) {
+    case 16: return GemmCfg<FMT, 16>::XST;
+    case 32: return GemmCfg<FMT, 32>::XST;
+    case 64: return GemmCfg<FMT, 64>::XST;
+    case 128: return GemmCfg<FMT, 128>::XST;
+    default:
+      if constexpr (FMT == FMT_FP8S) return GemmCfg<FMT, 128>::XST;
+      else return GemmCfg<FMT, 256>::XST;
   }
 }
 template <int FMT>
@@ -305,7 +322,10 @@ int smem_for(int bn) {
     case 16: return GemmCfg<FMT, 16>::SMEM;
     case 32: return GemmCfg<FMT, 32>::SMEM;
     case 64: return GemmCfg<FMT, 64>::SMEM;
-    default: return GemmCfg<FMT, 128>::SMEM;
+    case 128: return GemmCfg<FMT, 128>::SMEM;
+    default:
+      if constexpr (FMT == FMT_FP8S) return GemmCfg<FMT, 128>::SMEM;
+      else return GemmCfg<FMT, 256>::SMEM;
   }
 }
 template <int FMT>
@@ -314,6 +334,9 @@ cudaError_t set_attrs() {
   if (e == cudaSuccess) e = GemmLauncher<FMT, 32>::set_attr();
   if (e == cudaSuccess) e = GemmLauncher<FMT, 64>::set_attr();
   if (e == cudaSuccess) e = GemmLauncher<FMT, 128>::set_attr();
+  if constexpr (FMT != FMT_FP8S) {
+    if (e == cudaSuccess) e = GemmLauncher<FMT, 256>::set_attr();
+  }
   return e;
 }
 template <int FMT>
@@ -322,7 +345,10 @@ cudaError_t launch_fmt(int bn, const CUtensorMap& tm, const GemmParams& p, int g
     case 16: return GemmLauncher<FMT, 16>::launch(tm, p, grid, st);
     case 32: return GemmLauncher<FMT, 32>::launch(tm, p, grid, st);
     case 64: return GemmLauncher<FMT, 64>::launch(tm, p, grid, st);
-    default: return GemmLauncher<FMT, 128>::launch(tm, p, grid, st);
+    case 128: return GemmLauncher<FMT, 128>::launch(tm, p, grid, st);
+    default:
+      if constexpr (FMT != FMT_FP8S) return GemmLauncher<FMT, 256>::launch(tm, p, grid, st);
+      return cudaErrorInvalidValue;   // never planned: the fused static-FP8 tile holds at most 128 x rows
   }
 }
 
@@ -364,9 +390,25 @@ int cluster_capacity(dqgemm_s* h, int bn, int split) {
 // than SMs, the K range of each tile is split over the S CTAs of a cluster,
 // S the largest power of two (<= 8, <= k_stages) whose T * S CTAs are all
 // resident.
-void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
+// From 129 rows on, an x tile of 256 rows halves the weight dequantization
+// per FLOP (one N = 256 MMA per k-step); it is taken when it keeps at least
+// half the SMs busy and its waves of tiles cost no more than 5/4 of the
+// 128-row tiling's (the 128-row tile is bound by the unpack, about 5/4 of
+// its MMA time).  The fused static-FP8 kernel stays at 128 rows.
+int pick_bn(const dqgemm_s* h, int M, bool xq) {
+  int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  if (M > 128 && !(h->fmt == FMT_FP8S && !xq)) {
+    const long long sms = h->num_sms, nt = h->n_tiles;
+    const long long t256 = (M + 255) / 256 * nt, t128 = (M + 127) / 128 * nt;
+    const long long w256 = (t256 + sms - 1) / sms, w128 = (t128 + sms - 1) / sms;
+    if (2 * t256 >= sms && w256 * 256 * 4 <= w128 * 128 * 5) bn = 256;
+  }
+  return bn;
+}
+
+void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl, bool xq = false) {
   std::memset(pl, 0, sizeof(*pl));
-  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  const int bn = pick_bn(h, M, xq);
   pl->bn = bn;
   pl->m_tiles = (M + bn - 1) / bn;
   pl->n_tiles = h->n_tiles;
@@ -386,7 +428,9 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
   // the split is a power of two (<= 8, so it divides every bn): each rank
   // then owns bn / S whole columns of the tile in the reduction
   int split = 1;
-  if (force_split >= 1 && force_split <= 8) {
+  if (bn > 128) {
+    // whole tiles only
+  } else if (force_split >= 1 && force_split <= 8) {
     while (split * 2 <= std::min(force_split, h->k_stages)) split *= 2;
     if (split > 1 && cluster_capacity(h, bn, split) < T) split = 1;
   } else if (T < slots) {
@@ -398,12 +442,23 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl) {
   }
   pl->max_segments = split;
   pl->grid = split > 1 ? (int)(T * split) : (int)std::min<long long>(T, h->num_sms);
-  int st = 0, sm = 0;
-  DQ_FMT_SWITCH(h->fmt, st = stages_for<F>(bn); sm = smem_for<F>(bn));
+  int st = 0, sm = 0, xs = 0;
+  if (xq) {
+    st = stages_for<FMT_FP8SQ>(bn);
+    sm = smem_for<FMT_FP8SQ>(bn);
+    xs = xstages_for<FMT_FP8SQ>(bn);
+  } else {
+    DQ_FMT_SWITCH(h->fmt, st = stages_for<F>(bn); sm = smem_for<F>(bn); xs = xstages_for<F>(bn));
+  }
   pl->stages = st;
   pl->smem_bytes = sm;
   pl->workspace_bytes = 0;
   pl->weight_bytes = h->weight_bytes;
+  pl->x_stages = xs;
+  // the split gives rank q the stages [q*KS/S, (q+1)*KS/S); whole tiles give
+  // a CTA every ceil(T / grid)-th tile
+  pl->max_cta_stages = split > 1 ? (h->k_stages + split - 1) / split
+                                 : (int)((T + pl->grid - 1) / pl->grid) * h->k_stages;
 }
 
 dqgemm_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA; }
@@ -471,7 +526,7 @@ dqgemm_status dqgemm_destroy(dqgemm_handle h) {
   cudaFree(h->wchunks);
   cudaFree(h->col_scale);
   cudaFree(h->bias);
-  cudaFree(h->status);
+  if (h->status_host) cudaFreeHost(h->status_host);
   delete h;
   return DQ_OK;
 }
@@ -504,6 +559,7 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   h->k_stages = (K + STAGE_K - 1) / STAGE_K;
   h->n_tiles = (N + TILE_N - 1) / TILE_N;
   h->weight_bytes = (long long)(hp.size() + hs.size());
+  h->timeout_ns = timeout_ns();
   cudaGetDevice(&h->device);
   cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
 
@@ -526,12 +582,17 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   h->wchunk_bytes = chunks.size();
 
   cudaError_t e = cudaMalloc(&h->wchunks, chunks.size());
-  if (e == cudaSuccess) e = cudaMalloc(&h->status, sizeof(int));
+  // the status word lives in mapped pinned host memory: kernels store to it,
+  // the host reads it without synchronizing the device
+  if (e == cudaSuccess) e = cudaHostAlloc(&h->status_host, sizeof(int), cudaHostAllocMapped | cudaHostAllocPortable);
+  if (e == cudaSuccess) {
+    *h->status_host = 0;
+    e = cudaHostGetDevicePointer(reinterpret_cast<void**>(&h->status), h->status_host, 0);
+  }
   if (e == cudaSuccess && (fmt == FMT_FP8 || fmt == FMT_FP8S)) e = cudaMalloc(&h->col_scale, (size_t)N * 4);
   if (e == cudaSuccess && bias) e = cudaMalloc(&h->bias, (size_t)N * 2);
   if (e != cudaSuccess) { dqgemm_destroy(h); return DQ_ERR_ALLOC; }
   e = cudaMemcpy(h->wchunks, chunks.data(), chunks.size(), cudaMemcpyHostToDevice);
-  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int));
   if (e == cudaSuccess && h->col_scale) e = cudaMemcpy(h->col_scale, hs.data(), (size_t)N * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess && h->bias) e = cudaMemcpy(h->bias, bias, (size_t)N * 2, cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) { DQ_FMT_SWITCH(fmt, e = set_attrs<F>()); }
@@ -539,6 +600,12 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) { dqgemm_destroy(h); return DQ_ERR_CUDA; }
   *out = h;
+  return DQ_OK;
+}
+
+dqgemm_status dqgemm_set_wait_limit(dqgemm_handle h, long long timeout_ns_) {
+  if (!h || timeout_ns_ < 0) return DQ_ERR_INVALID_ARG;
+  h->timeout_ns = timeout_ns_ == 0 ? timeout_ns() : (unsigned long long)timeout_ns_;
   return DQ_OK;
 }
 
@@ -554,7 +621,7 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   if (yq && !(std::isfinite(s_out) && s_out > 0.f)) return DQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
   dqgemm_plan pl;
-  fill_plan(h, M, &pl);
+  fill_plan(h, M, &pl, xq);
   CUtensorMap tm;
   bool x3d = false;
   if (xq ? !make_q_map(&tm, x, M, h->K, pl.bn) : !make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
@@ -576,7 +643,8 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   p.tiles = pl.m_tiles * pl.n_tiles;
   p.split = pl.max_segments;
   p.x3d = x3d ? 1 : 0;
-  p.timeout_ns = timeout_ns();
+  p.timeout_ns = h->timeout_ns;
+  p.drain_ns = std::max(timeout_ns(), kDefaultTimeoutNs);
   cudaError_t e = cudaSuccess;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (xq) {
@@ -812,13 +880,9 @@ dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt_, const float* W, int
 
 dqgemm_status dqgemm_last_error(dqgemm_handle h) {
   if (!h) return DQ_ERR_INVALID_ARG;
-  if (cudaDeviceSynchronize() != cudaSuccess) return DQ_ERR_CUDA;
-  int v = 0;
-  if (cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DQ_ERR_CUDA;
-  if (v != 0) {
-    cudaMemset(h->status, 0, sizeof(int));
-    cudaDeviceSynchronize();
-  }
+  volatile int* w = h->status_host;
+  const int v = *w;
+  if (v != 0) *w = 0;
   return v == 0 ? DQ_OK : (dqgemm_status)v;
 }
 

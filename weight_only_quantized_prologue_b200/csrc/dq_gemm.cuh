@@ -52,7 +52,10 @@ struct GemmParams {
   int tiles;                     // n_tiles * m_tiles
   int split;                     // CTAs per tile (cluster size); 1 = whole tiles
   int x3d;                       // x map is 3-D {64, M, K/64}: one box per stage
-  unsigned long long timeout_ns;
+  unsigned long long timeout_ns;  // limit of the pipeline's waits
+  unsigned long long drain_ns;    // limit of the waits for this CTA's own copies, MMAs and received
+                                  // partials (never shorter than the default: leaving early would
+                                  // free shared or tensor memory that is still being written)
   uint8_t* yq;                   // if set: y goes out as e4m3 codes of bf16(y) / s_out
   float s_out;                   //   (the next static-FP8 layer's activation codes)
 };
@@ -85,27 +88,46 @@ struct GemmCfg {
   static constexpr int X_SLOT = align_up(X_BYTES, 1024) + align_up(Q_BYTES, 1024);
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);    // within an x slot
   static constexpr int W_SLOT = align_up(CHUNK, 1024);
-  static constexpr int XST = BN <= 32 ? 3 : 2;
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
-  static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : 200 * 1024;
-  static constexpr int WST_RAW = (SMEM_BUDGET - XST * X_SLOT - 3072) / W_SLOT;   // barriers, EPI, slack
+  static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : (BN <= 128 ? 200 * 1024 : 216 * 1024);
+  // split-K receive area: the S - 1 peers' partial columns this CTA owns,
+  // [peer slot][row][BN / S] fp32, at most 7/8 of a 128 x BN fp32 tile (S = 8),
+  // then one validity word per peer
+  // (256-row x tiles run whole tiles only: no receive area)
+  static constexpr int RECV_BYTES = BN >= 256 ? 0 : 7 * TILE_N * BN * 4 / 8;
+  static constexpr int RFLAG_BYTES = 64;
+  static constexpr int AVAIL = SMEM_BUDGET - RECV_BYTES - RFLAG_BYTES - 3072;   // barriers, EPI, slack
+  // The x ring is as deep as the budget allows while keeping three weight
+  // slots: a skinny split CTA (six 128-k stages at 32 x 3072 x 4096) then
+  // issues every x load of its k-range right after the grid-dependency wait.
+  static constexpr int XST = (AVAIL - 6 * X_SLOT >= 3 * W_SLOT)   ? 6
+                             : (AVAIL - 4 * X_SLOT >= 3 * W_SLOT) ? 4
+                             : (AVAIL - 3 * X_SLOT >= 3 * W_SLOT) ? 3
+                                                                  : 2;
+  static constexpr int WST_RAW = (AVAIL - XST * X_SLOT) / W_SLOT;
   static constexpr int WST = WST_RAW < 2 ? 2 : (WST_RAW > 8 ? 8 : WST_RAW);
   static constexpr int STAGES = WST;   // weight stages in flight (reported by the plan)
   static constexpr int X_RING_OFF = 0;
   static constexpr int W_RING_OFF = XST * X_SLOT;
+  static constexpr int RECV_OFF = W_RING_OFF + WST * W_SLOT;
+  static constexpr int RFLAG_OFF = RECV_OFF + RECV_BYTES;
   // TMEM: a ring of bf16 A operands (weights, one 128 x 128 stage each) and
   // the fp32 accumulators.  Two MMA-issuing threads (in different warps) each
   // own half of every stage's k-steps and an accumulator of their own: one
   // thread issues an MMA only every ~80 cycles, two issue in parallel.  The
   // epilogue adds the two accumulators in a fixed order.
-  static constexpr int ISSUERS = 2;
+  // (a 256-row x tile needs one issuer only: an N = 256 MMA keeps the tensor
+  // pipe busy for longer than a thread takes to issue the next)
+  static constexpr int ISSUERS = BN >= 256 ? 1 : 2;
+  // k-steps (of 16 bf16 / 32 e4m3) per stage each issuer takes
+  static constexpr int KK = (STATIC ? 4 : 8) / ISSUERS;
   static constexpr int A_STAGES = STATIC ? 0 : (BN == 64 ? 2 : 3);
   static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
   static constexpr int TMEM_COLS = pow2_at_least(A_COLS + ISSUERS * BN);
-  static constexpr int BAR_OFF = W_RING_OFF + WST * W_SLOT;
-  static constexpr int BAR_BYTES = 8 * 40;
+  static constexpr int BAR_OFF = RFLAG_OFF + RFLAG_BYTES;
+  static constexpr int BAR_BYTES = 8 * 64;
   // each epilogue thread's row factor and bias, parked in shared memory over
   // the main loop instead of holding registers: [2][256] fp32
   static constexpr int EPI_OFF = BAR_OFF + BAR_BYTES;
@@ -116,9 +138,10 @@ struct GemmCfg {
   // 11 x producer
   static constexpr int THREADS = 384;
   static_assert(A_COLS + ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
+  static_assert(!(STATIC && !XQ && BN > 128), "the fused static-FP8 tile holds at most 128 x rows");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");   // (two CTAs per SM need <= 113 KB)
-  static_assert(A_STAGES <= 3 && XST <= 3, "barrier arrays");
-  static_assert(XST * X_SLOT + WST * W_SLOT >= BN * TILE_N * 4, "split-K partial tile fits in the rings");
+  static_assert(A_STAGES <= 8 && XST <= 8 && WST <= 8, "barrier arrays");
+  static_assert(RECV_BYTES % 16 == 0 && RECV_OFF % 16 == 0, "16-byte st.async targets");
 };
 
 // The work of one CTA: a list of (tile, k_begin, k_end) segments.
@@ -249,28 +272,29 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint8_t* w_ring = smem + C::W_RING_OFF;
   uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);   // [8] weight chunk landed
   uint64_t* wempty = full_w + 8;          // [8] weight slot read (prologue, or MMAs for static FP8)
-  uint64_t* full_x = wempty + 8;          // [3] x tile landed
-  uint64_t* xempty = full_x + 3;          // [3] x slot read by the MMAs
-  uint64_t* aready = xempty + 3;          // [3] operand written: TMEM A slot (bf16) / e4m3 x (static, per x slot)
-  uint64_t* aempty = aready + 3;          // [3] TMEM A slot read by the MMAs
-  uint64_t* acc_full = aempty + 3;
+  uint64_t* full_x = wempty + 8;          // [8] x tile landed
+  uint64_t* xempty = full_x + 8;          // [8] x slot read by the MMAs
+  uint64_t* aready = xempty + 8;          // [8] operand written: TMEM A slot (bf16) / e4m3 x (static, per x slot)
+  uint64_t* aempty = aready + 8;          // [8] TMEM A slot read by the MMAs
+  uint64_t* acc_full = aempty + 8;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;        // [2], one per MMA issuer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* recv_bar = drain + 2;         // split-K: the peers' partials and flags have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);             // [S-1][128][BN/S]
+  uint32_t* rflag = reinterpret_cast<uint32_t*>(smem + C::RFLAG_OFF);     // [S-1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // wait control, rebuilt from kernel parameters at each wait so that it
   // holds no registers across the long loops
   const auto ctl = [&] { return WaitCtl{abort_flag, p.status, p.timeout_ns}; };
-  const auto ctl_no_abort = [&] { return WaitCtl{nullptr, p.status, p.timeout_ns}; };
+  const auto ctl_no_abort = [&] { return WaitCtl{nullptr, p.status, p.drain_ns}; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s) {
       mbar_init(&full_w[s], 1);
       mbar_init(&wempty[s], C::STATIC ? C::ISSUERS : 8);
-    }
-    for (int s = 0; s < 3; ++s) {
       mbar_init(&full_x[s], 1);
       mbar_init(&xempty[s], C::ISSUERS);
       mbar_init(&aready[s], 8);
@@ -280,6 +304,13 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     mbar_init(acc_empty, 8);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(recv_bar, 1);
+    if (p.split > 1) {
+      // every peer sends this CTA its partial of the columns this CTA owns
+      // plus one validity word, whether or not its own work succeeded
+      const int cmax = BN / p.split;
+      mbar_arrive_expect_tx(recv_bar, (uint32_t)((p.split - 1) * (TILE_N * cmax * 4 + 4)));
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -288,6 +319,9 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // split-K: no CTA sends into a peer before the peer's receive barrier is
+  // initialized (this barrier runs before the grid-dependency wait)
+  if (p.split > 1) cluster_sync();
   const uint32_t tmem = *tmem_slot;
   pdl_launch_dependents();   // the next call may start its own prologue now
 
@@ -363,13 +397,13 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     __syncwarp();
   } else if (warp == 1 || warp == 10) {
     // ------------------------------------------------------------ MMA issuers
-    if (lane == 0) {
+    if (lane == 0 && (warp == 1 || C::ISSUERS == 2)) {
       const int which = warp == 1 ? 0 : 1;   // k-steps [which*KK, (which+1)*KK) of each stage
-      constexpr int KK = C::STATIC ? 2 : 4;
+      constexpr int KK = C::KK;
       const uint32_t d_tmem = tmem + C::ACC_COL + which * BN;
       int ws = 0, xs = 0, as = 0;
       uint32_t wph = 0, xph = 0, aph = 0;
-      bool ok = true;
+      bool ok = true, issued = false;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
         if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl())) break;
         tc_fence_after();
@@ -378,11 +412,15 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           if constexpr (!C::STATIC) {
             if (!mbar_wait(&full_x[xs], xph, ctl()) || !mbar_wait(&aready[as], aph, ctl())) { ok = false; break; }
             tc_fence_after();
-            const uint32_t bx = xb + which * BN * 128;
             const uint32_t a_tmem = tmem + as * (STAGE_K / 2) + which * KK * 8;
 #pragma unroll
-            for (int kk = 0; kk < KK; ++kk)
-              mma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(bx + kk * 32), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < KK; ++kk) {
+              // k-step ks of the stage: 64-k box ks / 4 of the x slot, 32 bytes per k-step in its rows
+              const int ks = which * KK + kk;
+              const uint32_t bx = xb + (ks >> 2) * BN * 128 + (ks & 3) * 32;
+              mma_bf16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(bx), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            issued = true;
             tc_commit(&aempty[as]);
             if (++as == C::A_STAGES) {
               as = 0;
@@ -397,6 +435,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
             for (int kk = 0; kk < KK; ++kk)
               mma_f8_ss(d_tmem, sdesc_sw128(wb + kk * 32), sdesc_sw128(qb + kk * 32), C::IDESC,
                         (j > 0 || kk > 0) ? 1u : 0u);
+            issued = true;
             tc_commit(&wempty[ws]);
             if (++ws == C::WST) {
               ws = 0;
@@ -412,9 +451,13 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         if (!ok) break;
         tc_commit(acc_full);
       }
-      // all MMAs this thread issued must finish before TMEM is released
-      tc_commit(&drain[which]);
-      mbar_wait(&drain[which], 0, ctl_no_abort());
+      // all MMAs this thread issued must finish before TMEM is released (a
+      // commit with no MMA before it would never arrive: an issuer that gave
+      // up before its first MMA has nothing to drain)
+      if (issued) {
+        tc_commit(&drain[which]);
+        mbar_wait(&drain[which], 0, ctl_no_abort());
+      }
     }
     __syncwarp();
   } else {
@@ -425,7 +468,12 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     const int r = qd * 32 + lane;       // weight row in the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
     constexpr int HALF = BN / 2;
-    float acc[HALF];
+    // 256-row x tiles stream the accumulator out in chunks (its 128 columns
+    // per thread would not fit in registers); smaller tiles hold it whole
+    constexpr bool CHUNKED = BN > 128;
+    float acc[CHUNKED ? 1 : HALF];
+#pragma unroll
+    for (int i = 0; i < (CHUNKED ? 1 : HALF); ++i) acc[i] = 0.f;
     float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);   // [2][256]: this thread's slots only
     const int et = threadIdx.x - 64;
     int tile = 0;
@@ -501,6 +549,37 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // ---- epilogue of this tile
       if (!mbar_wait_warp(acc_full, t & 1, ctl())) { ok = false; break; }
       tc_fence_after();
+      if constexpr (CHUNKED) {
+        // one accumulator (one issuer): 32 columns at a time, the TMEM
+        // accumulator released after the last load, then that chunk stored
+        const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
+        const float e_sig = epi[et], e_bias = epi[256 + et];
+#pragma unroll 1
+        for (int c32 = 0; c32 < HALF / 32; ++c32) {
+          float a[32];
+          tmem_ld32(tmem + lane_base + C::ACC_COL + h * HALF + c32 * 32, a);
+          tmem_wait_ld();
+          if (c32 == HALF / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          if (n_row < p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int m = m_tile * BN + h * HALF + c32 * 32 + i;
+              if (m < p.M) {
+                if constexpr (!QOUT)
+                  p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(a[i], e_sig, e_bias));
+                else
+                  p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(a[i], e_sig, e_bias));
+              }
+            }
+          }
+        }
+        have_acc = true;
+        continue;
+      } else {
 #pragma unroll
       for (int c8 = 0; c8 < HALF / 8; ++c8) {
         float a1[8];
@@ -535,62 +614,82 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           }
         }
       }
+      }   // !CHUNKED
     }
     if (!ok) *abort_flag = 1;
 
-    if (p.split > 1) {
-      // ---- cluster split-K.  Every CTA writes its whole partial tile into
-      // its own (now idle) rings as [column][row] fp32; after one cluster
-      // barrier, rank q reads the tile's columns [q*BN/S, (q+1)*BN/S) of all
-      // S partials (its peers' through distributed shared memory) and adds
-      // them in rank order (deterministic).  A second cluster barrier keeps
-      // every CTA alive until its peers have read its partial.  Every
-      // epilogue warp takes part even after an abort.
+    if constexpr (!CHUNKED) if (p.split > 1) {
+      // ---- cluster split-K by push.  Rank q owns the tile's columns
+      // [q*BN/S, (q+1)*BN/S).  Every CTA sends each peer d its partial of
+      // d's columns with st.async straight into d's receive area (whose
+      // barrier counts the bytes), plus one word saying whether the partial
+      // is valid; it sends even after an abort, so that every receive
+      // completes.  The threads holding this CTA's own columns then add the
+      // S partials in rank order (deterministic) and store y if all S were
+      // valid.  No CTA leaves before every CTA of the cluster has received
+      // everything sent to it (the closing cluster barrier below).
       const int S = p.split;
       const int q = (int)cluster_rank();
       const int cmax = BN / S;
-      const bool good = ok && have_acc;
-      float* part = reinterpret_cast<float*>(smem);   // [BN][TILE_N] over both rings; all MMAs are done
-      if (good) {
+      named_barrier_sync(1, 256);                      // every epilogue warp has its verdict in abort_flag
+      const uint32_t good = *abort_flag ? 0u : 1u;
+      if (cmax >= 4) {
 #pragma unroll
-        for (int i = 0; i < HALF; ++i) part[(h * HALF + i) * TILE_N + r] = acc[i];
-      }
-      cluster_sync();   // every partial of the cluster is written (release / acquire)
-      const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
-      const float e_sig = epi[et], e_bias = epi[256 + et];
-      const bool all_good = good && !*abort_flag;
-      // This thread's HALF values are the S partials of columns
-      // c0 + h + 2 * ci, ci < cmax / 2 (S * cmax / 2 = HALF): all the loads
-      // are issued first, then each column is added in rank order.
-      const int c0 = q * cmax;
-      const int lg_s = __ffs(S) - 1;   // S is a power of two
-      float v[HALF];
-#pragma unroll
-      for (int i = 0; i < HALF; ++i) {
-        const int pr = i & (S - 1);
-        const int c = c0 + h + 2 * (i >> lg_s);
-        v[i] = pr == q ? part[c * TILE_N + r] : ld_dsmem_f32(part + c * TILE_N + r, (uint32_t)pr);
-      }
-      float sum = 0.f;
-      if constexpr (!QOUT) {
-#pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const int pr = i & (S - 1);
-          sum = pr == 0 ? v[i] : sum + v[i];
-          if (pr == S - 1) {
-            const int m = m_tile * BN + c0 + h + 2 * (i >> lg_s);
-            if (all_good && n_row < p.N && m < p.M)
-              p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
+        for (int i = 0; i < HALF; i += 4) {
+          const int c = h * HALF + i;                  // this thread's columns c .. c+3 lie in one owner's range
+          const int d = c / cmax;
+          if (d != q) {
+            const int slot = q < d ? q : q - 1;
+            const uint32_t dst = dsmem_addr(recv + (slot * TILE_N + r) * cmax + (c - d * cmax), (uint32_t)d);
+            st_async_v4(dst, acc[i], acc[i + 1], acc[i + 2], acc[i + 3], dsmem_addr(recv_bar, (uint32_t)d));
           }
         }
       } else {
 #pragma unroll
+        for (int i = 0; i < HALF; i += 2) {
+          const int c = h * HALF + i;
+          const int d = c / cmax;
+          if (d != q) {
+            const int slot = q < d ? q : q - 1;
+            const uint32_t dst = dsmem_addr(recv + (slot * TILE_N + r) * cmax + (c - d * cmax), (uint32_t)d);
+            st_async_v2(dst, acc[i], acc[i + 1], dsmem_addr(recv_bar, (uint32_t)d));
+          }
+        }
+      }
+      if (et == 0) {
+        for (int d = 0; d < S; ++d) {
+          if (d == q) continue;
+          const int slot = q < d ? q : q - 1;
+          st_async_u32(dsmem_addr(rflag + slot, (uint32_t)d), good, dsmem_addr(recv_bar, (uint32_t)d));
+        }
+      }
+      // the threads that hold this CTA's own columns reduce them
+      if (h == (q * cmax) / HALF) {
+        const WaitCtl rx_ctl{nullptr, p.status, 2 * p.drain_ns};
+        int rx = 1;
+        if (lane == 0) rx = mbar_wait_cluster(recv_bar, 0, rx_ctl) ? 1 : 0;
+        rx = __shfl_sync(0xFFFFFFFFu, rx, 0);
+        if (rx) mbar_try_wait_cluster(recv_bar, 0);
+        bool all_good = good && rx;
+        for (int sl = 0; sl < S - 1; ++sl) all_good = all_good && rflag[sl] != 0u;
+        const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
+        const float e_sig = epi[et], e_bias = epi[256 + et];
+#pragma unroll
         for (int i = 0; i < HALF; ++i) {
-          const int pr = i & (S - 1);
-          sum = pr == 0 ? v[i] : sum + v[i];
-          if (pr == S - 1) {
-            const int m = m_tile * BN + c0 + h + 2 * (i >> lg_s);
-            if (all_good && n_row < p.N && m < p.M) p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(sum, e_sig, e_bias));
+          const int c = h * HALF + i;
+          if (c / cmax != q) continue;
+          const int cl = c - q * cmax;
+          float sum = 0.f;
+          for (int pr = 0; pr < S; ++pr) {
+            const float v = pr == q ? acc[i] : recv[((pr < q ? pr : pr - 1) * TILE_N + r) * cmax + cl];
+            sum = pr == 0 ? v : sum + v;
+          }
+          const int m = m_tile * BN + c;
+          if (all_good && n_row < p.N && m < p.M) {
+            if constexpr (!QOUT)
+              p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
+            else
+              p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(sum, e_sig, e_bias));
           }
         }
       }
@@ -598,13 +697,12 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   }
 
   __syncwarp();
+  // split-K: every thread of the cluster arrives once its part is done (the
+  // reducing threads after their receive completed), so past this barrier
+  // no st.async into any CTA of the cluster is still in flight
   if (p.split > 1) {
-    // the non-epilogue warps take the first cluster barrier here; then no CTA
-    // leaves before its peers have read its partial (their reads completed
-    // before they arrive, so the arrive needs no release)
-    if (warp < 2 || warp >= 10) cluster_sync();
-    cluster_arrive_relaxed();
-    cluster_wait();
+    cluster_arrive_release();
+    cluster_wait_acquire();
   }
   tc_fence_before();
   __syncthreads();
