@@ -91,12 +91,12 @@ struct GemmCfg {
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
   static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : (BN <= 128 ? 200 * 1024 : 216 * 1024);
-  // split-K receive area: the S - 1 peers' partial columns this CTA owns,
-  // [peer slot][row][BN / S] fp32, at most 7/8 of a 128 x BN fp32 tile (S = 8),
-  // then one validity word per peer
-  // (256-row x tiles run whole tiles only: no receive area)
-  static constexpr int RECV_BYTES = BN >= 256 ? 0 : 7 * TILE_N * BN * 4 / 8;
-  static constexpr int RFLAG_BYTES = 64;
+  // split-K receive area: the S partials (its own included) of the columns
+  // this CTA owns, [rank][row][BN / S] fp32 = one 128 x BN fp32 tile, then
+  // one validity word per (rank, 32 rows) (256-row x tiles run whole tiles
+  // only: none)
+  static constexpr int RECV_BYTES = BN >= 256 ? 0 : TILE_N * BN * 4;
+  static constexpr int RFLAG_BYTES = 128;   // [8 ranks][4 row quadrants]
   static constexpr int AVAIL = SMEM_BUDGET - RECV_BYTES - RFLAG_BYTES - 3072;   // barriers, EPI, slack
   // The x ring is as deep as the budget allows while keeping three weight
   // slots: a skinny split CTA (six 128-k stages at 32 x 3072 x 4096) then
@@ -282,10 +282,11 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint64_t* recv_bar = drain + 2;         // split-K: the peers' partials and flags have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);             // [S-1][128][BN/S]
-  uint32_t* rflag = reinterpret_cast<uint32_t*>(smem + C::RFLAG_OFF);     // [S-1]
+  float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);             // [S][128][BN/S]
+  uint32_t* rflag = reinterpret_cast<uint32_t*>(smem + C::RFLAG_OFF);     // [S][4]: sender rank, row quadrant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  bool arrived = false;   // split-K: this thread has arrived at the closing cluster barrier (warp-uniform)
   // wait control, rebuilt from kernel parameters at each wait so that it
   // holds no registers across the long loops
   const auto ctl = [&] { return WaitCtl{abort_flag, p.status, p.timeout_ns}; };
@@ -307,9 +308,10 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     mbar_init(recv_bar, 1);
     if (p.split > 1) {
       // every peer sends this CTA its partial of the columns this CTA owns
-      // plus one validity word, whether or not its own work succeeded
+      // plus one validity word per 32 rows, whether or not its own work
+      // succeeded
       const int cmax = BN / p.split;
-      mbar_arrive_expect_tx(recv_bar, (uint32_t)((p.split - 1) * (TILE_N * cmax * 4 + 4)));
+      mbar_arrive_expect_tx(recv_bar, (uint32_t)((p.split - 1) * (TILE_N * cmax * 4 + 4 * 4)));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -622,74 +624,114 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // ---- cluster split-K by push.  Rank q owns the tile's columns
       // [q*BN/S, (q+1)*BN/S).  Every CTA sends each peer d its partial of
       // d's columns with st.async straight into d's receive area (whose
-      // barrier counts the bytes), plus one word saying whether the partial
-      // is valid; it sends even after an abort, so that every receive
-      // completes.  The threads holding this CTA's own columns then add the
-      // S partials in rank order (deterministic) and store y if all S were
+      // barrier counts the bytes).  Each sending warp adds one word saying
+      // whether its 32 rows are valid (it held its accumulator); it sends
+      // even after an abort, so that every receive completes.  The threads
+      // holding this CTA's own columns then add the S partials in rank order
+      // (deterministic) and store y where every partial of their rows was
       // valid.  No CTA leaves before every CTA of the cluster has received
       // everything sent to it (the closing cluster barrier below).
       const int S = p.split;
       const int q = (int)cluster_rank();
       const int cmax = BN / S;
-      named_barrier_sync(1, 256);                      // every epilogue warp has its verdict in abort_flag
-      const uint32_t good = *abort_flag ? 0u : 1u;
+      const uint32_t good = (ok && have_acc) ? 1u : 0u;   // warp-uniform
+      const int lg_cmax = __ffs(cmax) - 1;                 // cmax is a power of two
+      // (compact code: this part runs once per call, its instructions are
+      // fetched cold, and each one costs more than its work)
       if (cmax >= 4) {
 #pragma unroll
         for (int i = 0; i < HALF; i += 4) {
           const int c = h * HALF + i;                  // this thread's columns c .. c+3 lie in one owner's range
-          const int d = c / cmax;
-          if (d != q) {
-            const int slot = q < d ? q : q - 1;
-            const uint32_t dst = dsmem_addr(recv + (slot * TILE_N + r) * cmax + (c - d * cmax), (uint32_t)d);
-            st_async_v4(dst, acc[i], acc[i + 1], acc[i + 2], acc[i + 3], dsmem_addr(recv_bar, (uint32_t)d));
-          }
+          const int d = c >> lg_cmax;
+          float* slot = recv + (q * TILE_N + r) * cmax + (c & (cmax - 1));
+          if (d == q)
+            *reinterpret_cast<float4*>(slot) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+          else
+            st_async_v4(dsmem_addr(slot, (uint32_t)d), acc[i], acc[i + 1], acc[i + 2], acc[i + 3],
+                        dsmem_addr(recv_bar, (uint32_t)d));
         }
       } else {
 #pragma unroll
         for (int i = 0; i < HALF; i += 2) {
           const int c = h * HALF + i;
-          const int d = c / cmax;
-          if (d != q) {
-            const int slot = q < d ? q : q - 1;
-            const uint32_t dst = dsmem_addr(recv + (slot * TILE_N + r) * cmax + (c - d * cmax), (uint32_t)d);
-            st_async_v2(dst, acc[i], acc[i + 1], dsmem_addr(recv_bar, (uint32_t)d));
-          }
+          const int d = c >> lg_cmax;
+          float* slot = recv + (q * TILE_N + r) * cmax + (c & (cmax - 1));
+          if (d == q)
+            *reinterpret_cast<float2*>(slot) = make_float2(acc[i], acc[i + 1]);
+          else
+            st_async_v2(dsmem_addr(slot, (uint32_t)d), acc[i], acc[i + 1], dsmem_addr(recv_bar, (uint32_t)d));
         }
       }
-      if (et == 0) {
-        for (int d = 0; d < S; ++d) {
-          if (d == q) continue;
-          const int slot = q < d ? q : q - 1;
-          st_async_u32(dsmem_addr(rflag + slot, (uint32_t)d), good, dsmem_addr(recv_bar, (uint32_t)d));
-        }
+      // this warp's validity word, to every peer it sent rows to: the owners
+      // of the columns in half h, rflag[sender rank][row quadrant]
+      if (lane == 0) {
+        for (int d = (h * HALF) >> lg_cmax; d < ((h + 1) * HALF) >> lg_cmax; ++d)
+          if (d != q) st_async_u32(dsmem_addr(rflag + q * 4 + qd, (uint32_t)d), good, dsmem_addr(recv_bar, (uint32_t)d));
       }
-      // the threads that hold this CTA's own columns reduce them
+      // the threads that hold this CTA's own columns reduce them: row r,
+      // columns [q*cmax, (q+1)*cmax), the S partials in rank order (this
+      // thread wrote its own partial into slot q above)
       if (h == (q * cmax) / HALF) {
         const WaitCtl rx_ctl{nullptr, p.status, 2 * p.drain_ns};
         int rx = 1;
         if (lane == 0) rx = mbar_wait_cluster(recv_bar, 0, rx_ctl) ? 1 : 0;
         rx = __shfl_sync(0xFFFFFFFFu, rx, 0);
         if (rx) mbar_try_wait_cluster(recv_bar, 0);
+        // nothing more lands in this CTA: arrive at the closing barrier now,
+        // so that it never waits on this CTA's stores
+        cluster_arrive_relaxed();
+        arrived = true;
         bool all_good = good && rx;
-        for (int sl = 0; sl < S - 1; ++sl) all_good = all_good && rflag[sl] != 0u;
-        const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
-        const float e_sig = epi[et], e_bias = epi[256 + et];
+        for (int pr = 0; pr < S; ++pr) all_good = all_good && (pr == q || rflag[pr * 4 + qd] != 0u);
+        const int n_row = (tile / p.m_tiles) * TILE_N + r, m0 = (tile % p.m_tiles) * BN + q * cmax;
+        if (all_good && n_row < p.N) {
+          const float e_sig = epi[et], e_bias = epi[256 + et];
+          const float* row = recv + r * cmax;          // partial of rank pr at row[pr * TILE_N * cmax]
+          const int rstride = TILE_N * cmax;
+          // columns in chunks of (at most) 8: the S partials of a chunk are
+          // vector loads, added in rank order
+          const int cw = cmax < 8 ? cmax : 8;
+#pragma unroll 1
+          for (int c0 = 0; c0 < cmax && m0 + c0 < p.M; c0 += cw) {
+            float v[8];
+            const float* src = row + c0;
+            if (cw >= 4) {
+              const float4 a = *reinterpret_cast<const float4*>(src);
+              v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+              if (cw == 8) {
+                const float4 b = *reinterpret_cast<const float4*>(src + 4);
+                v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+              }
+            } else {
+              const float2 a = *reinterpret_cast<const float2*>(src);
+              v[0] = a.x; v[1] = a.y;
+            }
+#pragma unroll 1
+            for (int pr = 1; pr < S; ++pr) {
+              src += rstride;
+              if (cw >= 4) {
+                const float4 a = *reinterpret_cast<const float4*>(src);
+                v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+                if (cw == 8) {
+                  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+                  v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+                }
+              } else {
+                const float2 a = *reinterpret_cast<const float2*>(src);
+                v[0] += a.x; v[1] += a.y;
+              }
+            }
 #pragma unroll
-        for (int i = 0; i < HALF; ++i) {
-          const int c = h * HALF + i;
-          if (c / cmax != q) continue;
-          const int cl = c - q * cmax;
-          float sum = 0.f;
-          for (int pr = 0; pr < S; ++pr) {
-            const float v = pr == q ? acc[i] : recv[((pr < q ? pr : pr - 1) * TILE_N + r) * cmax + cl];
-            sum = pr == 0 ? v : sum + v;
-          }
-          const int m = m_tile * BN + c;
-          if (all_good && n_row < p.N && m < p.M) {
-            if constexpr (!QOUT)
-              p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(sum, e_sig, e_bias));
-            else
-              p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(sum, e_sig, e_bias));
+            for (int i = 0; i < 8; ++i) {
+              const int m = m0 + c0 + i;
+              if (i < cw && m < p.M) {
+                const size_t o = (size_t)m * p.N + n_row;
+                if constexpr (!QOUT)
+                  p.y[o] = __float2bfloat16_rn(fmaf(v[i], e_sig, e_bias));
+                else
+                  p.yq[o] = out_code(p, fmaf(v[i], e_sig, e_bias));
+              }
+            }
           }
         }
       }
@@ -697,12 +739,13 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   }
 
   __syncwarp();
-  // split-K: every thread of the cluster arrives once its part is done (the
-  // reducing threads after their receive completed), so past this barrier
-  // no st.async into any CTA of the cluster is still in flight
+  // split-K: every thread of the cluster arrives once (the reducing threads
+  // as soon as their receive completed, every other thread when its part is
+  // done), so past this barrier no st.async into any CTA of the cluster is
+  // still in flight and no sender leaves with one outstanding
   if (p.split > 1) {
-    cluster_arrive_release();
-    cluster_wait_acquire();
+    if (!arrived) cluster_arrive_relaxed();
+    cluster_wait();
   }
   tc_fence_before();
   __syncthreads();
