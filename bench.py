@@ -65,10 +65,15 @@ def algorithmic_bytes(fmt, M, K, N, bias=True):
     return w + M * K * 2 + M * N * 2 + (N * 2 if bias else 0)
 
 
+# the sources that define the GEMM kernel itself (its launch parameters
+# included); the other kernels and the host code do not change its traffic
+GEMM_SOURCES = ("dq_common.cuh", "dq_gemm.cuh", "dq_layout.h")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_only_quantized_prologue_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in GEMM_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -700,10 +705,10 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 
 
-def run_ncu_case(fmt):
-    """Eight back-to-back calls of one format at the step's Linear shape,
-    rotating over four weight sets: the case the committed ncu captures take
-    (one launch, after four warm ones)."""
+def run_ncu_case(fmt, M=LM, K=LK, N=LN):
+    """Eight back-to-back calls of one format, rotating over four weight
+    sets: the case the committed ncu captures take (one launch, after four
+    warm ones).  Default shape: the step's Linear at M=32."""
     import torch
 
     import weight_only_quantized_prologue_b200 as dq
@@ -712,16 +717,17 @@ def run_ncu_case(fmt):
     torch.cuda.set_device(0)
     layers = []
     for r in range(4):
-        x, w, b = synthetic.linear_inputs(LM, LK, LN, seed=r)
-        layers.append(dq.QuantizedLinear.from_float(fmt, w.cuda(), b.cuda()))
-    xc = x.cuda()
-    y = torch.empty((LM, LN), dtype=torch.bfloat16, device="cuda")
+        _, w, b = synthetic.linear_inputs(1, K, N, seed=r)
+        layers.append(dq.QuantizedLinear.from_float(fmt, w.cuda(), None if fmt == "fp8_static" else b.cuda(),
+                                                    act_scale=0.011))
+    xc = synthetic.activations(M, K, seed=1).cuda()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     for i in range(8):
         layers[i % 4](xc, out=y)
     torch.cuda.synchronize()
     for l in layers:
         assert l.last_error() == 0, "device-side wait timed out"
-    print(json.dumps({"ncu_case": fmt, "M": LM, "K": LK, "N": LN, "plan": layers[0].plan(LM)}), flush=True)
+    print(json.dumps({"ncu_case": fmt, "M": M, "K": K, "N": N, "plan": layers[0].plan(M)}), flush=True)
 
 
 def run_sweep(args):
@@ -797,9 +803,10 @@ def main():
     ap.add_argument("--sweep-m", default="1,16,32,128,1024,4096")
     ap.add_argument("--sweep-kn", default="4096x4096,4096x14336,14336x4096")
     ap.add_argument("--sweep-formats", default="int4,nvfp4,mxfp4,fp8,fp8_static")
-    ap.add_argument("--ncu-case", choices=list(LIN_FORMATS), default=None,
-                    help="small profiling case: 8 plain launches of one format at the step's shape "
-                         "(4 weight sets, no graphs, no timing) for an ncu capture")
+    ap.add_argument("--ncu-case", choices=list(LIN_FORMATS) + ["fp8_static", "int4_asym"], default=None,
+                    help="small profiling case: 8 plain launches of one format (4 weight sets, no graphs, "
+                         "no timing) for an ncu capture; the step's shape unless --ncu-shape is given")
+    ap.add_argument("--ncu-shape", default=None, help="MxKxN of the profiling case, e.g. 4096x4096x4096")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -811,7 +818,8 @@ def main():
         run_sweep(args)
         return
     if args.ncu_case:
-        run_ncu_case(args.ncu_case)
+        shape = [int(v) for v in args.ncu_shape.split("x")] if args.ncu_shape else [LM, LK, LN]
+        run_ncu_case(args.ncu_case, *shape)
         return
 
     if args.impl == "reference":

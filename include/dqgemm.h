@@ -36,8 +36,10 @@
  *     later call on it must be made with that device current, with x, y and
  *     the stream on that device (not checked: the launch goes to the current
  *     device).
- *   - The run entry points keep no host state between calls, so one handle
- *     may be run from several host threads and streams at once.
+ *   - The run entry points keep no host state between calls apart from a
+ *     small cache of the activation tensor maps they encode (a map depends
+ *     only on x, M and the tile; the cache is locked), so one handle may be
+ *     run from several host threads and streams at once.
  *     dqgemm_destroy must not overlap any other call on the same handle, nor
  *     any of its kernels still in flight.
  *

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "dq_aux.cuh"
@@ -30,6 +31,19 @@ struct dqgemm_s {
   long long weight_bytes = 0;       // canonical packed + scale bytes
   int max_clusters[4][9] = {};      // co-resident clusters per (BN index, cluster size), 0 = unknown
   unsigned long long timeout_ns = 0;  // limit of the kernels' pipeline waits
+  // activation tensor maps already encoded, by (x, M, tile rows, e4m3 input):
+  // encoding one costs host time on every call, and layers see the same
+  // few activation buffers again and again
+  struct MapEntry {
+    const void* x = nullptr;
+    int M = 0, bn = 0;
+    bool xq = false, x3d = false;
+    CUtensorMap map;
+  };
+  static constexpr int kMaps = 8;
+  MapEntry maps[kMaps];
+  int next_map = 0;
+  std::mutex maps_mu;               // run entry points may be called from several threads
 };
 
 namespace {
@@ -624,7 +638,31 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   fill_plan(h, M, &pl, xq);
   CUtensorMap tm;
   bool x3d = false;
-  if (xq ? !make_q_map(&tm, x, M, h->K, pl.bn) : !make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
+  {
+    // a map encodes only (x, M, K, tile rows): a cached one for the same
+    // key is the map this call would encode
+    std::lock_guard<std::mutex> lock(h->maps_mu);
+    bool hit = false;
+    for (const auto& e : h->maps) {
+      if (e.x == x && e.M == M && e.bn == pl.bn && e.xq == xq) {
+        tm = e.map;
+        x3d = e.x3d;
+        hit = true;
+        break;
+      }
+    }
+    if (!hit) {
+      if (xq ? !make_q_map(&tm, x, M, h->K, pl.bn) : !make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
+      auto& e = h->maps[h->next_map];
+      h->next_map = (h->next_map + 1) % dqgemm_s::kMaps;
+      e.x = x;
+      e.M = M;
+      e.bn = pl.bn;
+      e.xq = xq;
+      e.x3d = x3d;
+      e.map = tm;
+    }
+  }
   GemmParams p;
   p.wchunks = h->wchunks;
   p.col_scale = h->col_scale;
