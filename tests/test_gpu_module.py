@@ -85,3 +85,38 @@ def test_layer_rejects_bad_tensors_before_launch():
     torch.cuda.synchronize()
     assert lin.last_error() == 0 and y.shape == (8, 128)
     lin.close()
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4", "fp8", "int4_asym", "fp8_static"])
+def test_quantized_module_matches_oracle(fmt):
+    """The pages' flow end to end against the fp64 oracle: a bf16
+    nn.Linear(3072, 512) quantized in place by quantize_, called on x with
+    leading dims; the reference quantizes the same weight with the oracle's
+    own recipe and multiplies in fp64 ("Define a linear model and quantize
+    weights to ..." on each weight-only page; static FP8 with its calibrated
+    scale, "Define a small two-layer Linear model")."""
+    import numpy as np
+
+    from oracle import linear as L
+
+    from gpu_util import bf16_values, check_close, static_effective_x
+
+    torch.manual_seed(7)
+    model = torch.nn.Sequential(torch.nn.Linear(3072, 512)).to(device="cuda", dtype=torch.bfloat16)
+    W = model[0].weight.detach().float().cpu().numpy().astype(np.float64)
+    b = bf16_values(model[0].bias.detach())
+    x = synthetic.activations(2 * 20, 3072, seed=12).cuda().view(2, 20, 3072)
+    scales = None
+    if fmt == "fp8_static":
+        scales = M.calibrate_static_fp8(model, [synthetic.activations(32, 3072, seed=s).cuda() for s in range(1, 4)])
+    M.quantize_(model, fmt, act_scales=scales)
+    with torch.no_grad():
+        y = model(x)
+    torch.cuda.synchronize()
+    assert model[0].layer.last_error() == 0
+    base = "fp8" if fmt == "fp8_static" else fmt
+    st = L.quantize_pack(base, W)
+    wdq = L.dequant_exact(base, st["packed"], st["scales"], st["global_scale"])
+    xv = bf16_values(x.view(-1, 3072))
+    x_eff = static_effective_x(xv, scales["0"]) if fmt == "fp8_static" else xv
+    check_close(bf16_values(y.view(-1, 512)), L.linear_ref(x_eff, wdq, b), x_eff, wdq)

@@ -96,6 +96,27 @@ def test_quantize_act_fp8_bit_exact():
     assert np.array_equal(q.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("M,K,offset", [(5, 19, 0), (129, 4096, 0), (3, 272, 1), (64, 1000, 3)])
+def test_quantize_act_fp8_vector_tail_and_unaligned(M, K, offset):
+    # 16 elements per thread where x and q are 16-byte aligned, element-wise
+    # for the tail (M*K not a multiple of 16) and for unaligned buffers
+    rng = np.random.default_rng(M + K)
+    x = torch.from_numpy(rng.normal(0, 5, (M, K)).astype(np.float32)).to(torch.bfloat16)
+    x.view(-1)[::97] = 0.0
+    x.view(-1)[1::89] = -0.0
+    s_x = float(np.float32(0.0371))
+    xb = torch.zeros(M * K + 8, dtype=torch.bfloat16, device="cuda")
+    xb[offset:offset + M * K] = x.view(-1).cuda()
+    qb = torch.full((M * K + 16,), 0xEE, dtype=torch.uint8, device="cuda")
+    lib = dq._native.lib()
+    st = lib.dqgemm_quantize_act_fp8(xb.data_ptr() + 2 * offset, M, K, s_x, qb.data_ptr() + offset, None)
+    assert st == 0
+    torch.cuda.synchronize()
+    got = qb.cpu().numpy()
+    assert np.array_equal(got[offset:offset + M * K], L.quantize_act_fp8(bf16_values(x), s_x).reshape(-1))
+    assert (got[:offset] == 0xEE).all() and (got[offset + M * K:] == 0xEE).all()
+
+
 # -- GEMM parity -----------------------------------------------------------
 
 SHAPES = [(1, 256, 128), (3, 384, 256), (17, 512, 384), (33, 1024, 640), (64, 256, 1152),

@@ -730,9 +730,26 @@ dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream) {
 dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x, void* q, void* stream) {
   if (!x || !q || M < 1 || K < 1 || !(std::isfinite(s_x) && s_x > 0.f)) return DQ_ERR_INVALID_ARG;
   const long long count = (long long)M * K;
-  const int blocks = (int)std::min<long long>((count + 255) / 256, 148 * 8);
-  act_quant_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x), count, s_x, static_cast<uint8_t*>(q));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  uint8_t* qb = static_cast<uint8_t*>(q);
+  // 16 elements per thread where both buffers are 16-byte aligned, the
+  // element-wise kernel for the tail (or for everything otherwise)
+  long long done = 0;
+  if (aligned16(x) && aligned16(q)) {
+    const long long groups = count / 16;
+    if (groups > 0) {
+      const int blocks = (int)std::min<long long>((groups + 255) / 256, 148 * 8);
+      act_quant16_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(xb), groups, s_x,
+                                                 reinterpret_cast<uint4*>(qb));
+      done = groups * 16;
+    }
+  }
+  if (done < count) {
+    const long long rest = count - done;
+    const int blocks = (int)std::min<long long>((rest + 255) / 256, 148 * 8);
+    act_quant_kernel<<<blocks, 256, 0, s>>>(xb + done, rest, s_x, qb + done);
+  }
   return cuda_err(cudaGetLastError());
 }
 
