@@ -4,8 +4,9 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
 the pages' nn.Linear(3072, 4096) on x[32, 3072] in each weight-only format
 (INT4 g128, NVFP4, MXFP4, FP8 E4M3 per-channel) plus the static-FP8 page's
-two-layer 256->512->128 model on x[32, 256] -- six dqgemm_run calls.  The
-metric is microseconds per call (step time / 6), lower is better.
+two-layer 256->512->128 model on x[32, 256] -- six Linear layers, run as
+four dqgemm_run calls and one dqgemm_run_static_mlp.  The metric is
+microseconds per Linear layer (step time / 6), lower is better.
 
 Weights rotate round-robin over R independent weight sets whose packed bytes
 total at least 3x the L2 size, so every call streams its weight from HBM.
@@ -37,9 +38,11 @@ UNIT = "µs/call"
 LIN_FORMATS = ("int4", "nvfp4", "mxfp4", "fp8")
 LM, LK, LN = 32, 3072, 4096
 MLP_IN, MLP_HID, MLP_OUT = 256, 512, 128
-CALLS_PER_STEP = len(LIN_FORMATS) + 2
+CALLS_PER_STEP = len(LIN_FORMATS) + 2          # Linear layers (DQ-GEMMs) per step
+LAUNCHES_PER_STEP = len(LIN_FORMATS) + 1       # the static MLP's two layers run in one launch
 WORKLOAD = ("Linear(3072->4096), x[32,3072] bf16, in INT4-g128 / NVFP4 / MXFP4 / FP8-WO + "
-            "static-FP8 MLP 256->512->128 (no bias), x[32,256]; 6 calls per step")
+            "static-FP8 MLP 256->512->128 (no bias), x[32,256]; 6 Linear layers per step in 5 launches "
+            "(the MLP's two layers in one); value = step time / 6 layers")
 
 
 # ---------------------------------------------------------------------------
@@ -195,23 +198,23 @@ class WeightSet:
         self.mlp2 = dq.QuantizedLinear.from_float("fp8_static", w2.float(), None, act_scale=s2)
         self.xm = synthetic.activations(LM, MLP_IN, seed=1000 * idx + 8).to(dev)
         self.y = {f: torch.empty((LM, LN), dtype=torch.bfloat16, device=dev) for f in LIN_FORMATS}
-        self.h = torch.empty((LM, MLP_HID), dtype=torch.bfloat16, device=dev)
         self.ym = torch.empty((LM, MLP_OUT), dtype=torch.bfloat16, device=dev)
         self.weight_bytes = sum(l.plan(LM)["weight_bytes"] for l in self.layers.values()) + \
             self.mlp1.plan(LM)["weight_bytes"] + self.mlp2.plan(LM)["weight_bytes"]
 
-    def calls(self):
-        """(name, layer, x, y) in step order."""
-        out = [(f, self.layers[f], self.x, self.y[f]) for f in LIN_FORMATS]
-        out.append(("fp8_static_l1", self.mlp1, self.xm, self.h))
-        out.append(("fp8_static_l2", self.mlp2, self.h, self.ym))
+    def calls(self, dq, stream=None):
+        """(name, launch) in step order: the four Linear layers, then the
+        two-layer static MLP as one launch."""
+        out = [(f, (lambda f=f: self.layers[f](self.x, out=self.y[f], stream=stream))) for f in LIN_FORMATS]
+        out.append(("fp8_static_mlp", lambda: dq.static_mlp(self.mlp1, self.mlp2, self.xm, out=self.ym,
+                                                             stream=stream)))
         return out
 
-    def step(self, torch, events=None):
-        for i, (name, layer, x, y) in enumerate(self.calls()):
+    def step(self, torch, dq, events=None):
+        for i, (name, launch) in enumerate(self.calls(dq)):
             if events is not None:
                 events[i][0].record()
-            layer(x, out=y)
+            launch()
             if events is not None:
                 events[i][1].record()
 
@@ -229,7 +232,7 @@ def run_ours(args, rank, world, local_rank):
     R = max(2, math.ceil(3 * l2 / first.weight_bytes))
     sets = [first] + [WeightSet(i, torch, dq, synthetic) for i in range(1, R)]
     for s in sets:                       # first calls allocate split-K workspaces
-        s.step(torch)
+        s.step(torch, dq)
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
@@ -238,18 +241,18 @@ def run_ours(args, rank, world, local_rank):
         for s in sets:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                s.step(torch)
+                s.step(torch, dq)
             graphs.append(g)
         # a second graph family with CUDA events around every call, for the
         # per-kernel durations behind the roofline figure
         n_ev = 2 * R
         ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-               for _ in range(CALLS_PER_STEP)]
+               for _ in range(LAUNCHES_PER_STEP)]
               for _ in range(n_ev)]
         g_ev = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_ev, stream=stream):
             for i in range(n_ev):
-                sets[i % R].step(torch, events=ev[i])
+                sets[i % R].step(torch, dq, events=ev[i])
     torch.cuda.synchronize()
 
     def barrier():
@@ -288,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
         # per-kernel durations (events inside the graph)
         g_ev.replay()
         torch.cuda.synchronize()
-    names = [c[0] for c in first.calls()]
+    names = [c[0] for c in first.calls(dq)]
     per_call = {n: statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(n_ev)) * 1000.0
                 for j, n in enumerate(names)}
 
@@ -299,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     # end-to-end through the public API with host buffers: per call, pinned
     # host x -> device, dqgemm_run, device y -> pinned host
     e2e_steps = max(3, min(args.steps, 200))
-    e2e = EndToEnd(torch, sets, stream)
+    e2e = EndToEnd(torch, dq, sets, stream)
     h2d, d2h = e2e.h2d_bytes, e2e.d2h_bytes
     e2e.run(3)
     torch.cuda.synchronize()
@@ -311,6 +314,7 @@ def run_ours(args, rank, world, local_rank):
 
     single = single_launch_us(torch, sets, stream)
     b2b = {f: back_to_back_us(torch, sets, stream, f) for f in LIN_FORMATS}
+    b2b_mlp = back_to_back_us(torch, sets, stream, "fp8_static_mlp", dq=dq)
     wide = None if args.no_wide else wide_block(torch, dq, synthetic, stream, measured_peaks())
 
     for s in sets:
@@ -338,8 +342,8 @@ def run_ours(args, rank, world, local_rank):
         per_format[n] = {"us": round(b2b[n], 3), "GB/s": round(ab / (b2b[n] * 1e-6) / 1e9, 1),
                          "frac_hbm": round(ab / (b2b[n] * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
                          "isolated_us": round(per_call[n], 3)}
-    per_format["fp8_static_l1"] = {"isolated_us": round(per_call["fp8_static_l1"], 3)}
-    per_format["fp8_static_l2"] = {"isolated_us": round(per_call["fp8_static_l2"], 3)}
+    per_format["fp8_static_mlp"] = {"us": round(b2b_mlp, 3), "isolated_us": round(per_call["fp8_static_mlp"], 3),
+                                    "layers": 2}
     result = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": False,
@@ -352,7 +356,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline,
         "e2e": {"value": round(job_us_per_call(e2e_ms, e2e_steps, CALLS_PER_STEP, world), 4), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps * CALLS_PER_STEP,
+        "gpu_launches": args.steps * LAUNCHES_PER_STEP,
         "clocks": clocks,
         "single_launch_us": single,
         "wide": wide,
@@ -360,7 +364,7 @@ def run_ours(args, rank, world, local_rank):
     return result, sets
 
 
-def back_to_back_us(torch, sets, stream, fmt, calls=240):
+def back_to_back_us(torch, sets, stream, fmt, calls=240, dq=None):
     """Device time per call of one format's calls back to back (a CUDA graph
     of `calls` calls rotating over the weight sets, as consecutive layers of
     a decode step run): the per-format figure of the metric.  Median of 5
@@ -370,7 +374,10 @@ def back_to_back_us(torch, sets, stream, fmt, calls=240):
         with torch.cuda.graph(g, stream=stream):
             for i in range(calls):
                 st = sets[i % len(sets)]
-                st.layers[fmt](st.x, out=st.y[fmt], stream=stream)
+                if fmt == "fp8_static_mlp":
+                    dq.static_mlp(st.mlp1, st.mlp2, st.xm, out=st.ym, stream=stream)
+                else:
+                    st.layers[fmt](st.x, out=st.y[fmt], stream=stream)
         g.replay()
         stream.synchronize()
         t = []
@@ -476,12 +483,16 @@ class EndToEnd:
     IN = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static_l1")     # calls fed from the host
     OUT = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static_l2")    # results read back
 
-    def __init__(self, torch, sets, stream):
-        self.torch, self.sets, self.compute = torch, sets, stream
+    def __init__(self, torch, dq, sets, stream):
+        self.torch, self.dq, self.sets, self.compute = torch, dq, sets, stream
         self.up, self.down = torch.cuda.Stream(), torch.cuda.Stream()
-        calls = {n: (layer, x, y) for n, layer, x, y in sets[0].calls()}
-        self.in_shapes = [tuple(calls[n][1].shape) for n in self.IN]
-        self.out_shapes = [tuple(calls[n][2].shape) for n in self.OUT]
+        s0 = sets[0]
+        xs = {f: s0.x for f in LIN_FORMATS}
+        xs["fp8_static_l1"] = s0.xm
+        ys = {f: s0.y[f] for f in LIN_FORMATS}
+        ys["fp8_static_l2"] = s0.ym
+        self.in_shapes = [tuple(xs[n].shape) for n in self.IN]
+        self.out_shapes = [tuple(ys[n].shape) for n in self.OUT]
         n_in = sum(a * b for a, b in self.in_shapes)
         n_out = sum(a * b for a, b in self.out_shapes)
         self.h2d_bytes, self.d2h_bytes = 2 * n_in, 2 * n_out
@@ -489,13 +500,13 @@ class EndToEnd:
         # host: each weight set's own inputs, packed; results per buffer
         self.h_in = []
         for st in sets:
-            c = {n: x for n, _, x, _ in st.calls()}
+            c = {f: st.x for f in LIN_FORMATS}
+            c["fp8_static_l1"] = st.xm
             self.h_in.append(torch.cat([c[n].reshape(-1) for n in self.IN]).cpu().pin_memory())
         nb = self.NB
         self.h_out = [torch.empty(n_out, dtype=bf).pin_memory() for _ in range(nb)]
         self.d_in = [torch.empty(n_in, dtype=bf, device="cuda") for _ in range(nb)]
         self.d_out = [torch.empty(n_out, dtype=bf, device="cuda") for _ in range(nb)]
-        self.h1 = [torch.empty_like(sets[0].h) for _ in range(nb)]
         # per-call operand views into each packed buffer, made once
         self.vin = [dict(zip(self.IN, self._views(self.d_in[b], self.in_shapes))) for b in range(nb)]
         self.vout = [dict(zip(self.OUT, self._views(self.d_out[b], self.out_shapes))) for b in range(nb)]
@@ -529,8 +540,8 @@ class EndToEnd:
                 self.compute.wait_event(self.ev["down"][b])       # step i-NB's results are home
             for f in LIN_FORMATS:
                 st.layers[f](xin[f], out=yout[f], stream=self.compute)
-            st.mlp1(xin["fp8_static_l1"], out=self.h1[b], stream=self.compute)
-            st.mlp2(self.h1[b], out=yout["fp8_static_l2"], stream=self.compute)
+            self.dq.static_mlp(st.mlp1, st.mlp2, xin["fp8_static_l1"], out=yout["fp8_static_l2"],
+                               stream=self.compute)
             self.ev["done"][b].record(self.compute)
             with torch.cuda.stream(self.down):
                 self.down.wait_event(self.ev["done"][b])

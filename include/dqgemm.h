@@ -162,6 +162,28 @@ dqgemm_status dqgemm_run_quantized_out(dqgemm_handle h, const void* x, int M, vo
 dqgemm_status dqgemm_run_fp8_static_quantized_out(dqgemm_handle h, const void* q, int M, void* q_out,
                                                   float s_out, void* stream);
 
+/* The static page's two-layer model in one launch ("TorchAO Static FP8
+ * Quantization (Linear)", "Define a small two-layer Linear model" and the
+ * Q -> DQ -> GEMM -> Q -> DQ -> GEMM chain of its "Graph after export"):
+ *     h = bf16(layer1(x)),  y = bf16(layer2(e4m3(h / s_x2)))
+ * with l1, l2 DQ_FP8_STATIC handles (s_x2 is l2's activation scale, each
+ * layer's bias added if its handle has one).  Layer 1's output never leaves
+ * the chip: CTA q of a thread-block cluster computes hidden units
+ * [128q, 128q+128) over all of K, quantizes them into layer 2's operand in
+ * shared memory, multiplies them by layer 2's matching k-slice, and the
+ * cluster adds the slices in rank order (deterministic).
+ * x: device bf16 [M, K1]; y: device bf16 [M, N2]; h_out: NULL or device bf16
+ * [M, N1] receiving layer 1's output (for checks; y does not depend on it).
+ * Requirements: l2's K equals l1's N; N1 = 128 * S with S = 2, 4 or 8
+ * (256, 512 or 1024 hidden units); N2 <= 128; both handles on the current device (DQ_ERR_INVALID_ARG or
+ * DQ_ERR_UNSUPPORTED otherwise); 16-byte aligned buffers.  Layer 1 sums
+ * over K in one CTA, so h can differ in the last bit from a separate
+ * dqgemm_run of l1 (which may split K); everything else is the same
+ * arithmetic as two dqgemm_run calls.  Device-side timeouts are reported
+ * through dqgemm_last_error(l1). */
+dqgemm_status dqgemm_run_static_mlp(dqgemm_handle l1, dqgemm_handle l2, const void* x, int M,
+                                    void* h_out, void* y, void* stream);
+
 /* Release the handle and its device memory.  Synchronizes the device (the
  * CUDA runtime's cudaFree does so in any case); no kernel of the handle may
  * still be queued or running. */

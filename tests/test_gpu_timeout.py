@@ -59,3 +59,28 @@ def test_wait_limit_rejects_bad_arguments():
         assert lib.dqgemm_set_wait_limit(h, 0) == dq._native.DQ_OK
     finally:
         dq.dqgemm_destroy(h)
+
+
+def test_one_launch_mlp_wait_limit_expires_then_context_recovers():
+    # the two-layer static MLP in one launch takes its wait limit from layer 1
+    w1, w2 = synthetic.mlp_weights(seed=8)
+    l1 = dq.QuantizedLinear.from_float("fp8_static", w1.float().cuda(), None, act_scale=0.009)
+    l2 = dq.QuantizedLinear.from_float("fp8_static", w2.float().cuda(), None, act_scale=0.004)
+    try:
+        x = synthetic.activations(32, 256, seed=9).cuda()
+        y = torch.full((32, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dq.dqgemm_set_wait_limit(l1.handle, 1)
+        dq.static_mlp(l1, l2, x, out=y)
+        torch.cuda.synchronize()
+        assert l1.last_error() == dq._native.DQ_ERR_TIMEOUT
+        assert torch.isnan(y.float()).all(), "an aborted call wrote output"
+        dq.dqgemm_set_wait_limit(l1.handle, 0)
+        y2 = dq.static_mlp(l1, l2, x)
+        y3 = l2(l1(x))
+        torch.cuda.synchronize()
+        assert l1.last_error() == 0 and l2.last_error() == 0
+        err = (y2.float() - y3.float()).norm() / y3.float().norm()
+        assert err < 2e-2, err          # the same model computed by two launches
+    finally:
+        l1.close()
+        l2.close()

@@ -27,6 +27,7 @@ from ._native import (  # noqa: F401
     dqgemm_run_fp8_static_quantized,
     dqgemm_run_fp8_static_quantized_out,
     dqgemm_run_quantized_out,
+    dqgemm_run_static_mlp,
     dqgemm_selftest_timeout,
     dqgemm_set_wait_limit,
     dqgemm_status_string,
@@ -66,6 +67,30 @@ def _fits(t, cols, dtype, rows=None, device=None):
 def _storage_bytes(fmt, K, N):
     ps, pd, ss, sd = storage_shapes(fmt, K, N)
     return (int(_np.prod(ps)) * _np.dtype(pd).itemsize, int(_np.prod(ss)) * _np.dtype(sd).itemsize)
+
+
+def static_mlp(l1, l2, x, out=None, h_out=None, stream=None):
+    """The static-FP8 two-layer model y = l2(l1(x)) in one launch
+    (dqgemm_run_static_mlp): l1, l2 are "fp8_static" QuantizedLinear layers
+    with l2.K == l1.N, l1.N in {256, 512, 1024}, l2.N <= 128; x bf16
+    [M, l1.K] on their device.  Returns y (``out``, allocated if None);
+    ``h_out`` (bf16 [M, l1.N]) receives layer 1's output if given."""
+    import torch
+
+    if l1.fmt != "fp8_static" or l2.fmt != "fp8_static":
+        raise ValueError("static_mlp needs two fp8_static layers")
+    if l2.K != l1.N:
+        raise ValueError(f"layer 2 takes {l2.K} inputs, layer 1 gives {l1.N}")
+    if l2.device != l1.device:
+        raise ValueError("both layers must live on the same device")
+    M = l1._check_x(x, torch.bfloat16)
+    out = l2._out(out, M, torch.bfloat16, x.device)
+    if h_out is not None:
+        _require(h_out, "h_out", shape=(M, l1.N), dtype=torch.bfloat16, device=x.device)
+    if M == 0:
+        return out
+    dqgemm_run_static_mlp(l1.handle, l2.handle, x, M, h_out, out, stream)
+    return out
 
 
 class QuantizedLinear:

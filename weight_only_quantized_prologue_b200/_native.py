@@ -55,6 +55,7 @@ _SIGNATURES = {
     "dqgemm_selftest_timeout": [_I, _VP],
     "dqgemm_get_plan": [_VP, _I, ctypes.POINTER(Plan)],
     "dqgemm_set_wait_limit": [_VP, ctypes.c_longlong],
+    "dqgemm_run_static_mlp": [_VP, _VP, _VP, _I, _VP, _VP, _VP],
 }
 
 _lib = None
@@ -140,6 +141,11 @@ def dqgemm_run_quantized_out(h, x, M, q_out, s_out, stream=None):
 def dqgemm_run_fp8_static_quantized_out(h, q, M, q_out, s_out, stream=None):
     _check(lib().dqgemm_run_fp8_static_quantized_out(h, _ptr(q), int(M), _ptr(q_out), float(s_out),
                                                       _stream(stream)), "dqgemm_run_fp8_static_quantized_out")
+
+
+def dqgemm_run_static_mlp(l1, l2, x, M, h_out, y, stream=None):
+    _check(lib().dqgemm_run_static_mlp(l1, l2, _ptr(x), int(M), _ptr(h_out), _ptr(y), _stream(stream)),
+           "dqgemm_run_static_mlp")
 
 
 def dqgemm_destroy(h):

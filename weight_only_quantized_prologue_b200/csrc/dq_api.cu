@@ -248,7 +248,9 @@ struct GemmLauncher {
   using C = GemmCfg<FMT, BN>;
   static cudaError_t set_attr() {
     cudaError_t e = set_attr_q<false>();
-    if (e == cudaSuccess) e = set_attr_q<true>();
+    if constexpr (FMT != FMT_MLP) {
+      if (e == cudaSuccess) e = set_attr_q<true>();
+    }
     return e;
   }
   template <bool QOUT>
@@ -288,8 +290,12 @@ struct GemmLauncher {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attrs[2];
     config(cfg, attrs, grid, p.split, st);
-    return p.yq ? cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, true>, tm, p)
-                : cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, false>, tm, p);
+    if constexpr (FMT == FMT_MLP) {
+      return cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, false>, tm, p);
+    } else {
+      return p.yq ? cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, true>, tm, p)
+                  : cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, false>, tm, p);
+    }
   }
   static int max_active_clusters(int split) {
     cudaLaunchConfig_t cfg;
@@ -475,6 +481,30 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl, bool xq = false) {
                                  : (int)((T + pl->grid - 1) / pl->grid) * h->k_stages;
 }
 
+// The activation tensor map for (x, M, tile rows, e4m3 input), from the
+// handle's cache or freshly encoded.  A map encodes only those and K, so a
+// cached one for the same key is the map this call would encode.
+bool x_map(dqgemm_s* h, const void* x, int M, int bn, bool xq, CUtensorMap* tm, bool* x3d) {
+  std::lock_guard<std::mutex> lock(h->maps_mu);
+  for (const auto& e : h->maps) {
+    if (e.x == x && e.M == M && e.bn == bn && e.xq == xq) {
+      *tm = e.map;
+      *x3d = e.x3d;
+      return true;
+    }
+  }
+  if (xq ? !make_q_map(tm, x, M, h->K, bn) : !make_x_map(tm, x, M, h->K, bn, x3d)) return false;
+  auto& e = h->maps[h->next_map];
+  h->next_map = (h->next_map + 1) % dqgemm_s::kMaps;
+  e.x = x;
+  e.M = M;
+  e.bn = bn;
+  e.xq = xq;
+  e.x3d = *x3d;
+  e.map = *tm;
+  return true;
+}
+
 dqgemm_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA; }
 
 // Codes the canonical storage may hold (the packers produce nothing else):
@@ -611,6 +641,9 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   if (e == cudaSuccess && h->bias) e = cudaMemcpy(h->bias, bias, (size_t)N * 2, cudaMemcpyDeviceToDevice);
   if (e == cudaSuccess) { DQ_FMT_SWITCH(fmt, e = set_attrs<F>()); }
   if (e == cudaSuccess && fmt == FMT_FP8S) e = set_attrs<FMT_FP8SQ>();
+  if (e == cudaSuccess && fmt == FMT_FP8S) e = GemmLauncher<FMT_MLP, 16>::set_attr();
+  if (e == cudaSuccess && fmt == FMT_FP8S) e = GemmLauncher<FMT_MLP, 32>::set_attr();
+  if (e == cudaSuccess && fmt == FMT_FP8S) e = GemmLauncher<FMT_MLP, 64>::set_attr();
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) { dqgemm_destroy(h); return DQ_ERR_CUDA; }
   *out = h;
@@ -638,32 +671,8 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   fill_plan(h, M, &pl, xq);
   CUtensorMap tm;
   bool x3d = false;
-  {
-    // a map encodes only (x, M, K, tile rows): a cached one for the same
-    // key is the map this call would encode
-    std::lock_guard<std::mutex> lock(h->maps_mu);
-    bool hit = false;
-    for (const auto& e : h->maps) {
-      if (e.x == x && e.M == M && e.bn == pl.bn && e.xq == xq) {
-        tm = e.map;
-        x3d = e.x3d;
-        hit = true;
-        break;
-      }
-    }
-    if (!hit) {
-      if (xq ? !make_q_map(&tm, x, M, h->K, pl.bn) : !make_x_map(&tm, x, M, h->K, pl.bn, &x3d)) return DQ_ERR_CUDA;
-      auto& e = h->maps[h->next_map];
-      h->next_map = (h->next_map + 1) % dqgemm_s::kMaps;
-      e.x = x;
-      e.M = M;
-      e.bn = pl.bn;
-      e.xq = xq;
-      e.x3d = x3d;
-      e.map = tm;
-    }
-  }
-  GemmParams p;
+  if (!x_map(h, x, M, pl.bn, xq, &tm, &x3d)) return DQ_ERR_CUDA;
+  GemmParams p{};
   p.wchunks = h->wchunks;
   p.col_scale = h->col_scale;
   p.bias = h->bias;
@@ -713,6 +722,54 @@ dqgemm_status dqgemm_run_fp8_static_quantized_out(dqgemm_handle h, const void* q
   if (!h) return DQ_ERR_INVALID_ARG;
   if (h->fmt != FMT_FP8S) return DQ_ERR_UNSUPPORTED;
   return run_gemm(h, q, true, M, q_out, true, s_out, stream);
+}
+
+dqgemm_status dqgemm_run_static_mlp(dqgemm_handle l1, dqgemm_handle l2, const void* x, int M, void* h_out, void* y,
+                                    void* stream) {
+  if (!l1 || !l2 || !x || !y || M < 1) return DQ_ERR_INVALID_ARG;
+  if (l1->fmt != FMT_FP8S || l2->fmt != FMT_FP8S) return DQ_ERR_UNSUPPORTED;
+  if (l2->K != l1->N || l1->N % TILE_N != 0) return DQ_ERR_INVALID_ARG;
+  const int S = l1->N / TILE_N;                 // cluster size: one hidden tile per CTA
+  // (the cluster's split-K hands each rank BN / S whole columns: S a power of two)
+  if ((S != 2 && S != 4 && S != 8) || l2->N > TILE_N || l1->device != l2->device) return DQ_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y) || (h_out && !aligned16(h_out))) return DQ_ERR_ALIGNMENT;
+  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+  const int m_tiles = (M + bn - 1) / bn;
+  CUtensorMap tm;
+  bool x3d = false;
+  if (!x_map(l1, x, M, bn, false, &tm, &x3d)) return DQ_ERR_CUDA;
+  GemmParams p{};
+  p.wchunks = l1->wchunks;
+  p.col_scale = l1->col_scale;
+  p.bias = l1->bias;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.status = l1->status;
+  p.sigma = l1->s_x;
+  p.s_x = l1->s_x;
+  p.s_out = l2->s_x;
+  p.M = M;
+  p.N = l1->N;
+  p.k_stages = l1->k_stages;
+  p.m_tiles = m_tiles;
+  p.tiles = S * m_tiles;
+  p.split = S;
+  p.x3d = x3d ? 1 : 0;
+  p.timeout_ns = l1->timeout_ns;
+  p.drain_ns = std::max(timeout_ns(), kDefaultTimeoutNs);
+  p.w2chunks = l2->wchunks;
+  p.col_scale2 = l2->col_scale;
+  p.bias2 = l2->bias;
+  p.h_out = static_cast<__nv_bfloat16*>(h_out);
+  p.N2 = l2->N;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int grid = S * m_tiles;
+  cudaError_t e;
+  switch (bn) {
+    case 16: e = GemmLauncher<FMT_MLP, 16>::launch(tm, p, grid, s); break;
+    case 32: e = GemmLauncher<FMT_MLP, 32>::launch(tm, p, grid, s); break;
+    default: e = GemmLauncher<FMT_MLP, 64>::launch(tm, p, grid, s); break;
+  }
+  return cuda_err(e);
 }
 
 dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream) {

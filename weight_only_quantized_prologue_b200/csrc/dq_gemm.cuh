@@ -58,6 +58,14 @@ struct GemmParams {
                                   // free shared or tensor memory that is still being written)
   uint8_t* yq;                   // if set: y goes out as e4m3 codes of bf16(y) / s_out
   float s_out;                   //   (the next static-FP8 layer's activation codes)
+  // two-layer static MLP (FMT_MLP): layer 1 is (wchunks, col_scale, bias,
+  // sigma = s_x) with N = hidden; its output is quantized with s_out and
+  // multiplied by layer 2 (w2chunks, col_scale2, bias2), N2 outputs
+  const uint8_t* w2chunks;
+  const float* col_scale2;
+  const __nv_bfloat16* bias2;
+  __nv_bfloat16* h_out;          // optional: layer 1's bf16 output [M, N]
+  int N2;
 };
 
 // the e4m3 code of an output for the next static-FP8 layer,
@@ -77,8 +85,9 @@ struct GemmCfg {
   // static FP8 with x quantized beforehand: x arrives as e4m3 [M, K] through
   // a 2-D u8 map (box 128 k x BN rows), straight into the operand buffer
   static constexpr bool XQ = (FMT == FMT_FP8SQ);
-  static constexpr bool STATIC = (FMT == FMT_FP8S) || XQ;
-  static constexpr int CHUNK = chunk_bytes(FMT);
+  static constexpr bool MLP = (FMT == FMT_MLP);
+  static constexpr bool STATIC = (FMT == FMT_FP8S) || XQ || MLP;
+  static constexpr int CHUNK = chunk_bytes(MLP ? FMT_FP8S : FMT);
   static constexpr int X_BYTES = XQ ? 0 : BN * 256;        // two 64-k blocks of BN rows x 128 B
   static constexpr int Q_BYTES = STATIC ? BN * 128 : 0;    // e4m3 x tile (static FP8)
   // Two rings: packed weight chunks (streamed from the start of the kernel;
@@ -97,7 +106,11 @@ struct GemmCfg {
   // only: none)
   static constexpr int RECV_BYTES = BN >= 256 ? 0 : TILE_N * BN * 4;
   static constexpr int RFLAG_BYTES = 128;   // [8 ranks][4 row quadrants]
-  static constexpr int AVAIL = SMEM_BUDGET - RECV_BYTES - RFLAG_BYTES - 3072;   // barriers, EPI, slack
+  // MLP: layer 2's weight chunk (its k-slice of this CTA's hidden columns)
+  // and layer 2's B operand, this CTA's hidden activations as e4m3 codes
+  static constexpr int W2_BYTES = MLP ? TILE_N * STAGE_K : 0;
+  static constexpr int B2_BYTES = MLP ? align_up(BN * STAGE_K, 1024) : 0;
+  static constexpr int AVAIL = SMEM_BUDGET - RECV_BYTES - RFLAG_BYTES - W2_BYTES - B2_BYTES - 3072;   // barriers, EPI, slack
   // The x ring is as deep as the budget allows while keeping three weight
   // slots: a skinny split CTA (six 128-k stages at 32 x 3072 x 4096) then
   // issues every x load of its k-range right after the grid-dependency wait.
@@ -112,6 +125,8 @@ struct GemmCfg {
   static constexpr int W_RING_OFF = XST * X_SLOT;
   static constexpr int RECV_OFF = W_RING_OFF + WST * W_SLOT;
   static constexpr int RFLAG_OFF = RECV_OFF + RECV_BYTES;
+  static constexpr int W2_OFF = align_up(RFLAG_OFF + RFLAG_BYTES, 1024);
+  static constexpr int B2_OFF = W2_OFF + W2_BYTES;
   // TMEM: a ring of bf16 A operands (weights, one 128 x 128 stage each) and
   // the fp32 accumulators.  Two MMA-issuing threads (in different warps) each
   // own half of every stage's k-steps and an accumulator of their own: one
@@ -125,8 +140,9 @@ struct GemmCfg {
   static constexpr int A_STAGES = STATIC ? 0 : (BN == 64 ? 2 : 3);
   static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
-  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + ISSUERS * BN);
-  static constexpr int BAR_OFF = RFLAG_OFF + RFLAG_BYTES;
+  static constexpr int ACC2_COL = ACC_COL + ISSUERS * BN;   // MLP: layer 2's accumulators
+  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN);
+  static constexpr int BAR_OFF = B2_OFF + B2_BYTES;
   static constexpr int BAR_BYTES = 8 * 64;
   // each epilogue thread's row factor and bias, parked in shared memory over
   // the main loop instead of holding registers: [2][256] fp32
@@ -137,7 +153,8 @@ struct GemmCfg {
   // warp 0 weight producer, 1 and 10 MMA issuers, 2..9 prologue/epilogue,
   // 11 x producer
   static constexpr int THREADS = 384;
-  static_assert(A_COLS + ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
+  static_assert(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
+  static_assert(!(MLP && BN > 64), "the MLP runs x tiles of at most 64 rows");
   static_assert(!(STATIC && !XQ && BN > 128), "the fused static-FP8 tile holds at most 128 x rows");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");   // (two CTAs per SM need <= 113 KB)
   static_assert(A_STAGES <= 8 && XST <= 8 && WST <= 8, "barrier arrays");
@@ -151,9 +168,18 @@ struct Work {
   __device__ int stages() const { return ntiles * (ke - kb); }
 };
 
+template <bool MLP>
 __device__ __forceinline__ Work cta_work(const GemmParams& p) {
   Work w;
-  if (p.split > 1) {
+  if (MLP) {
+    // rank q of the cluster computes layer 1's output tile q (all of K) for
+    // the cluster's m-tile; that tile is layer 2's k-slice q
+    w.first_tile = (int)cluster_rank() * p.m_tiles + (int)blockIdx.x / p.split;
+    w.tile_step = 1;
+    w.ntiles = 1;
+    w.kb = 0;
+    w.ke = p.k_stages;
+  } else if (p.split > 1) {
     const int q = (int)cluster_rank();
     w.first_tile = blockIdx.x / p.split;
     w.tile_step = 1;
@@ -280,7 +306,10 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;        // [2], one per MMA issuer
   uint64_t* recv_bar = drain + 2;         // split-K: the peers' partials and flags have landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_bar + 1);
+  uint64_t* full_w2 = recv_bar + 1;       // MLP: layer 2's weight chunk landed
+  uint64_t* b2ready = full_w2 + 1;        // MLP: layer 2's B operand (hidden codes) written
+  uint64_t* acc2_full = b2ready + 1;      // MLP: layer 2's accumulators complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc2_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);             // [S][128][BN/S]
   uint32_t* rflag = reinterpret_cast<uint32_t*>(smem + C::RFLAG_OFF);     // [S][4]: sender rank, row quadrant
@@ -306,6 +335,9 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(recv_bar, 1);
+    mbar_init(full_w2, 1);
+    mbar_init(b2ready, 8);
+    mbar_init(acc2_full, C::ISSUERS);
     if (p.split > 1) {
       // every peer sends this CTA its partial of the columns this CTA owns
       // plus one validity word per 32 rows, whether or not its own work
@@ -327,7 +359,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   const uint32_t tmem = *tmem_slot;
   pdl_launch_dependents();   // the next call may start its own prologue now
 
-  const Work wk = cta_work(p);
+  const Work wk = cta_work<C::MLP>(p);
   const int KS = p.k_stages;
   const int nst = wk.ke - wk.kb;   // stages per tile
   // (all ring positions are kept in counters: an integer division by a
@@ -338,6 +370,12 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     // Weights do not depend on earlier grids: they stream from the start, as
     // far ahead as the ring allows.
     if (lane == 0) {
+      if constexpr (C::MLP) {
+        // layer 2's weight chunk for this CTA's k-slice: its single output
+        // tile (N2 <= 128), stage q = the cluster rank
+        mbar_arrive_expect_tx(full_w2, C::CHUNK);
+        bulk_g2s(smem + C::W2_OFF, p.w2chunks + (size_t)cluster_rank() * C::CHUNK, C::CHUNK, full_w2);
+      }
       const int total = wk.stages();
       int ks = wk.kb, tile = wk.first_tile, ws = 0, it = 0;
       uint32_t wph = 0;
@@ -359,6 +397,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       // never leave with copies in flight: wait for the chunks issued last
       for (int i = it > C::WST ? it - C::WST : 0; i < it; ++i)
         mbar_wait(&full_w[i % C::WST], (i / C::WST) & 1, ctl_no_abort());
+      if constexpr (C::MLP) mbar_wait(full_w2, 0, ctl_no_abort());
     }
     __syncwarp();
   } else if (warp == 11) {
@@ -452,6 +491,21 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         }
         if (!ok) break;
         tc_commit(acc_full);
+      }
+      if constexpr (C::MLP) {
+        // layer 2 on this CTA's k-slice: A = layer 2's weight chunk, B = the
+        // hidden activations' e4m3 codes the epilogue warps wrote
+        if (ok && mbar_wait(full_w2, 0, ctl()) && mbar_wait(b2ready, 0, ctl())) {
+          tc_fence_after();
+          const uint32_t wb = smem_u32(smem + C::W2_OFF) + which * KK * 32;
+          const uint32_t bb = smem_u32(smem + C::B2_OFF) + which * KK * 32;
+          const uint32_t d2 = tmem + C::ACC2_COL + which * BN;
+#pragma unroll
+          for (int kk = 0; kk < KK; ++kk)
+            mma_f8_ss(d2, sdesc_sw128(wb + kk * 32), sdesc_sw128(bb + kk * 32), C::IDESC, kk > 0 ? 1u : 0u);
+          issued = true;
+          tc_commit(acc2_full);
+        }
       }
       // all MMAs this thread issued must finish before TMEM is released (a
       // commit with no MMA before it would never arrive: an issuer that gave
@@ -595,6 +649,49 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       have_acc = true;
+      if constexpr (C::MLP) {
+        // layer 1's epilogue: h = bf16(acc * s_x1 * s_w1[n] + b1[n]) for this
+        // thread's hidden unit n (tile q, row r) and the rows m of its half;
+        // the code e4m3(h / s_x2) is layer 2's B operand at (row m, k = r)
+        // (128-byte swizzled K-major rows), and h goes out if asked for
+        have_acc = false;
+        const int n1 = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
+        const float e_sig = epi[et], e_bias = epi[256 + et];
+        uint8_t* b2 = smem + C::B2_OFF;
+#pragma unroll
+        for (int i = 0; i < HALF; ++i) {
+          const int mm = h * HALF + i;
+          const float v = fmaf(acc[i], e_sig, e_bias);
+          const int m = m_tile * BN + mm;
+          if (p.h_out && m < p.M) p.h_out[(size_t)m * p.N + n1] = __float2bfloat16_rn(v);
+          b2[mm * 128 + (((r >> 4) ^ (mm & 7)) << 4) + (r & 15)] = out_code(p, v);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b2ready);
+        // layer 2's factors for its output row n2 = r (one tile of <= 128)
+        {
+          float e_sig2 = p.s_out, e_bias2 = 0.f;
+          if (r < p.N2) {
+            e_sig2 = p.s_out * ld_nc_f32(p.col_scale2 + r);
+            if (p.bias2) e_bias2 = ld_nc_bf16(p.bias2 + r);
+          }
+          epi[et] = e_sig2;
+          epi[256 + et] = e_bias2;
+        }
+        if (!mbar_wait_warp(acc2_full, 0, ctl())) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c8 = 0; c8 < HALF / 8; ++c8) {
+          float a1[8];
+          tmem_ld8(tmem + lane_base + C::ACC2_COL + h * HALF + c8 * 8, *reinterpret_cast<float(*)[8]>(acc + c8 * 8));
+          tmem_ld8(tmem + lane_base + C::ACC2_COL + BN + h * HALF + c8 * 8, a1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[c8 * 8 + i] += a1[i];
+        }
+        have_acc = true;
+      }
       // (no grid-dependency wait here: the producer's wait precedes the x
       // loads this accumulator depends on, so every earlier grid is done)
       if (p.split == 1) {
@@ -683,8 +780,11 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         arrived = true;
         bool all_good = good && rx;
         for (int pr = 0; pr < S; ++pr) all_good = all_good && (pr == q || rflag[pr * 4 + qd] != 0u);
-        const int n_row = (tile / p.m_tiles) * TILE_N + r, m0 = (tile % p.m_tiles) * BN + q * cmax;
-        if (all_good && n_row < p.N) {
+        // (MLP: layer 2's single output tile, N2 columns of y)
+        const int n_row = C::MLP ? r : (tile / p.m_tiles) * TILE_N + r;
+        const int n_out = C::MLP ? p.N2 : p.N;
+        const int m0 = (tile % p.m_tiles) * BN + q * cmax;
+        if (all_good && n_row < n_out) {
           const float e_sig = epi[et], e_bias = epi[256 + et];
           const float* row = recv + r * cmax;          // partial of rank pr at row[pr * TILE_N * cmax]
           const int rstride = TILE_N * cmax;
@@ -725,7 +825,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
             for (int i = 0; i < 8; ++i) {
               const int m = m0 + c0 + i;
               if (i < cw && m < p.M) {
-                const size_t o = (size_t)m * p.N + n_row;
+                const size_t o = (size_t)m * n_out + n_row;
                 if constexpr (!QOUT)
                   p.y[o] = __float2bfloat16_rn(fmaf(v[i], e_sig, e_bias));
                 else

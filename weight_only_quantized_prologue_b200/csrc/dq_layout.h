@@ -45,7 +45,10 @@ enum Fmt { FMT_INT4 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_FP8S = 4
            FMT_INT4A = 5,   // asymmetric INT4, per-group zero point
            // static FP8 GEMM fed with activations quantized beforehand (same
            // weight chunks as FMT_FP8S; a kernel variant, not a storage format)
-           FMT_FP8SQ = 8 };
+           FMT_FP8SQ = 8,
+           // the static-FP8 two-layer MLP in one launch (layer 1 in FP8S
+           // chunks, layer 2 likewise; a kernel variant)
+           FMT_MLP = 9 };
 
 constexpr int TILE_N = 128;      // output channels per tile (MMA M)
 constexpr int STAGE_K = 128;     // k per pipeline stage (= one INT4 group)
