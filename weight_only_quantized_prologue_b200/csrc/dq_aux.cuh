@@ -54,13 +54,13 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* wchunks, co
 __global__ void act_quant_kernel(const __nv_bfloat16* x, long long count, float s_x, uint8_t* q) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
        i += (long long)gridDim.x * blockDim.x) {
-    q[i] = e4m3_code(__fdiv_rn(__bfloat162float(x[i]), s_x));
+    q[i] = act_code(__bfloat162float(x[i]), s_x);
   }
 }
 
 // The same, 16 elements per thread: two 16-byte loads of bf16, one 16-byte
 // store of codes (x and q 16-byte aligned; `groups` = count / 16, the tail
-// goes to act_quant_kernel).  Each code is e4m3_code of the same quotient,
+// goes to act_quant_kernel).  Each code is act_code of the same value,
 // so the result is bit-identical with the element-wise kernel.
 __global__ void act_quant16_kernel(const uint4* x, long long groups, float s_x, uint4* q) {
   for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < groups;
@@ -74,8 +74,8 @@ __global__ void act_quant16_kernel(const uint4* x, long long groups, float s_x, 
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const uint32_t v = in[2 * w + k];
-        const uint32_t lo = e4m3_code(__fdiv_rn(__uint_as_float(v << 16), s_x));
-        const uint32_t hi = e4m3_code(__fdiv_rn(__uint_as_float(v & 0xFFFF0000u), s_x));
+        const uint32_t lo = act_code(__uint_as_float(v << 16), s_x);
+        const uint32_t hi = act_code(__uint_as_float(v & 0xFFFF0000u), s_x);
         word |= (lo | (hi << 8)) << (16 * k);
       }
       out[w] = word;

@@ -246,6 +246,13 @@ __device__ __forceinline__ uint8_t e4m3_code(float v) {
   return c;
 }
 
+// static-FP8 activation code of a value v (the Q node): e4m3(f32(v / s)),
+// IEEE division; a zero v gives its signed zero code without dividing
+// (the division is slow for a zero dividend, and exact either way)
+__device__ __forceinline__ uint8_t act_code(float v, float s) {
+  return v == 0.f ? (signbit(v) ? 0x80 : 0x00) : e4m3_code(__fdiv_rn(v, s));
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -72,7 +72,7 @@ struct GemmParams {
 // q = e4m3(f32(bf16(v)) / s_out): the code dqgemm_quantize_act_fp8 gives
 // for the bf16 output y = bf16(v)
 __device__ __forceinline__ uint8_t out_code(const GemmParams& p, float v) {
-  return e4m3_code(__fdiv_rn(__bfloat162float(__float2bfloat16_rn(v)), p.s_out));
+  return act_code(__bfloat162float(__float2bfloat16_rn(v)), p.s_out);
 }
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -276,7 +276,9 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
       for (int k = 0; k < 2; ++k) {
         const uint32_t w = in[2 * i + k];
         const float f0 = __uint_as_float(w << 16), f1 = __uint_as_float(w & 0xFFFF0000u);
-        const float2 qv = make_float2(__fdiv_rn(f0, s_x), __fdiv_rn(f1, s_x));
+        // (+-0 / s_x is +-0: no division, which is slow for a zero dividend;
+        // at one activation row 15 of a 16-row tile are the TMA's zero fill)
+        const float2 qv = make_float2(f0 == 0.f ? f0 : __fdiv_rn(f0, s_x), f1 == 0.f ? f1 : __fdiv_rn(f1, s_x));
         lohi[k] = (uint32_t)__nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
       }
       out[i] = lohi[0] | (lohi[1] << 16);
