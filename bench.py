@@ -36,6 +36,9 @@ if ROOT not in sys.path:
 METRIC = "DQ-GEMM µs/call; HBM GB/s (M≤128) & TFLOP/s (M≥1024) vs B200 roofline"
 UNIT = "µs/call"
 LIN_FORMATS = ("int4", "nvfp4", "mxfp4", "fp8")
+# FP4 x FP4 (native block-scaled MMA, activations quantized per call): timed
+# beside the step's formats at the same shape, not part of the step
+W4A4_FORMATS = ("w4a4_mxfp4", "w4a4_nvfp4")
 LM, LK, LN = 32, 3072, 4096
 MLP_IN, MLP_HID, MLP_OUT = 256, 512, 128
 CALLS_PER_STEP = len(LIN_FORMATS) + 2          # Linear layers (DQ-GEMMs) per step
@@ -52,7 +55,9 @@ WORKLOAD = ("Linear(3072->4096), x[32,3072] bf16, in INT4-g128 / NVFP4 / MXFP4 /
 
 def algorithmic_bytes(fmt, M, K, N, bias=True):
     """Bytes one call must move: packed weight + scales (+ zero points, +
-    global scale) + x + y + bias."""
+    global scale) + x + y + bias.  (W4A4: its weight storage format's bytes;
+    the quantized activation is an intermediate, not an input.)"""
+    fmt = {"w4a4_mxfp4": "mxfp4", "w4a4_nvfp4": "nvfp4"}.get(fmt, fmt)
     if fmt == "int4":
         w = N * K // 2 + N * (K // 128) * 2
     elif fmt == "int4_asym":
@@ -71,6 +76,12 @@ def algorithmic_bytes(fmt, M, K, N, bias=True):
 # the sources that define the GEMM kernel itself (its launch parameters
 # included); the other kernels and the host code do not change its traffic
 GEMM_SOURCES = ("dq_common.cuh", "dq_gemm.cuh", "dq_layout.h")
+
+
+def tensor_peak_ratio(fmt):
+    """The format's dense tensor-core peak over bf16's (nominal 4.5 / 2.25
+    PFLOP/s for FP8, 9 / 2.25 for FP4): the MMA each format runs."""
+    return 2.0 if fmt == "fp8_static" else 4.0 if fmt in W4A4_FORMATS else 1.0
 
 
 def kernel_source_hash():
@@ -313,8 +324,14 @@ def run_ours(args, rank, world, local_rank):
         e2e_ms = aggregate_max(e2e_ms)
 
     single = single_launch_us(torch, sets, stream)
-    b2b = {f: back_to_back_us(torch, sets, stream, f) for f in LIN_FORMATS}
-    b2b_mlp = back_to_back_us(torch, sets, stream, "fp8_static_mlp", dq=dq)
+    b2b, rotated_mb = {}, {}
+    for f in LIN_FORMATS + W4A4_FORMATS:
+        rot = FormatRotation(torch, dq, synthetic, f, l2)
+        b2b[f] = back_to_back_us(torch, stream, rot.launches(stream))
+        rotated_mb[f] = rot.rotated_mb
+        rot.close()
+    b2b_mlp = back_to_back_us(torch, stream, [
+        (lambda st=st: dq.static_mlp(st.mlp1, st.mlp2, st.xm, out=st.ym, stream=stream)) for st in sets])
     wide = None if args.no_wide else wide_block(torch, dq, synthetic, stream, measured_peaks())
 
     for s in sets:
@@ -326,7 +343,7 @@ def run_ours(args, rank, world, local_rank):
     # the roofline kernel: the slowest weight-only format of the step, timed
     # as a stream of back-to-back calls of that format (the per-format figure
     # of the metric; a call's average duration in that stream)
-    dom = max(b2b, key=b2b.get)
+    dom = max(LIN_FORMATS, key=b2b.get)
     alg = algorithmic_bytes(dom, LM, LK, LN)
     achieved = alg / (b2b[dom] * 1e-6) / 1e9
     traffic = ncu_traffic()
@@ -334,14 +351,19 @@ def run_ours(args, rank, world, local_rank):
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": (traffic or {}).get(dom), "algorithmic_bytes": alg,
                 "avg_launch_us": round(b2b[dom], 3),
-                "timing": "CUDA events around a graph of 240 back-to-back calls of this format",
+                "timing": (f"CUDA events around a graph of 240 back-to-back calls of this format, rotating "
+                           f"over {rotated_mb[dom]} MB of distinct weights (>= 3x L2)"),
                 "peak_source": f"{peaks['source']} (HBM copy)"}
     per_format = {}
-    for n in LIN_FORMATS:
+    for n in LIN_FORMATS + W4A4_FORMATS:
         ab = algorithmic_bytes(n, LM, LK, LN)
         per_format[n] = {"us": round(b2b[n], 3), "GB/s": round(ab / (b2b[n] * 1e-6) / 1e9, 1),
                          "frac_hbm": round(ab / (b2b[n] * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
-                         "isolated_us": round(per_call[n], 3)}
+                         "rotated_MB": rotated_mb[n]}
+        if n in per_call:
+            per_format[n]["isolated_us"] = round(per_call[n], 3)
+        else:
+            per_format[n]["note"] = "FP4 x FP4, x quantized per call (2 or 3 launches); not in the step"
     per_format["fp8_static_mlp"] = {"us": round(b2b_mlp, 3), "isolated_us": round(per_call["fp8_static_mlp"], 3),
                                     "layers": 2}
     result = {
@@ -364,20 +386,16 @@ def run_ours(args, rank, world, local_rank):
     return result, sets
 
 
-def back_to_back_us(torch, sets, stream, fmt, calls=240, dq=None):
-    """Device time per call of one format's calls back to back (a CUDA graph
-    of `calls` calls rotating over the weight sets, as consecutive layers of
-    a decode step run): the per-format figure of the metric.  Median of 5
+def back_to_back_us(torch, stream, launches, calls=240):
+    """Device time per call of a list of launches run back to back (a CUDA
+    graph of `calls` calls cycling over the list, as consecutive layers of a
+    decode step run): the per-format figure of the metric.  Median of 5
     replays."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g, stream=stream):
             for i in range(calls):
-                st = sets[i % len(sets)]
-                if fmt == "fp8_static_mlp":
-                    dq.static_mlp(st.mlp1, st.mlp2, st.xm, out=st.ym, stream=stream)
-                else:
-                    st.layers[fmt](st.x, out=st.y[fmt], stream=stream)
+                launches[i % len(launches)]()
         g.replay()
         stream.synchronize()
         t = []
@@ -392,6 +410,43 @@ def back_to_back_us(torch, sets, stream, fmt, calls=240, dq=None):
     return statistics.median(t)
 
 
+class FormatRotation:
+    """One format's Linear at the page shape as many distinct copies of one
+    packed weight as make >= 3x L2 (the back-to-back figure must not find
+    its weights in L2), with one x and one y."""
+
+    def __init__(self, torch, dq, synthetic, fmt, l2):
+        import numpy as np
+
+        x, w, b = synthetic.linear_inputs(LM, LK, LN, seed=4242)
+        w = w.cuda()
+        ps, pd, ss, sd = dq.storage_shapes(fmt, LK, LN)
+        tdt = {np.uint8: torch.uint8, np.uint16: torch.int16, np.float32: torch.float32}
+        packed = torch.empty(ps, dtype=tdt[pd], device="cuda")
+        scales = torch.empty(ss, dtype=tdt[sd], device="cuda")
+        g = dq.dqgemm_pack_device(fmt, w, packed, scales)
+        bias = b.cuda()
+        first = dq.QuantizedLinear(fmt, LK, LN, packed, scales, g, bias)
+        wb = first.plan(LM)["weight_bytes"]
+        R = max(2, math.ceil(3 * l2 / wb))
+        self.layers = [first] + [dq.QuantizedLinear(fmt, LK, LN, packed, scales, g, bias) for _ in range(R - 1)]
+        self.rotated_mb = round(R * wb / 2**20, 1)
+        self.x = x.cuda()
+        self.y = torch.empty((LM, LN), dtype=torch.bfloat16, device="cuda")
+        for l in self.layers:               # first calls (W4A4: allocate the activation workspace)
+            l(self.x, out=self.y)
+        torch.cuda.synchronize()
+
+    def launches(self, stream):
+        return [(lambda l=l: l(self.x, out=self.y, stream=stream)) for l in self.layers]
+
+    def close(self):
+        for l in self.layers:
+            assert l.last_error() == 0, "device-side wait timed out"
+            l.close()
+        self.layers = []
+
+
 WIDE_M, WIDE_K, WIDE_N = 4096, 4096, 4096
 
 
@@ -404,7 +459,7 @@ def wide_block(torch, dq, synthetic, stream, peaks, reps=24):
     M, K, N = WIDE_M, WIDE_K, WIDE_N
     xs = [synthetic.activations(M, K, seed=100 + i).cuda() for i in range(4)]
     ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
-    for fmt in list(LIN_FORMATS) + ["fp8_static"]:
+    for fmt in list(LIN_FORMATS) + ["fp8_static"] + list(W4A4_FORMATS):
         layers = []
         for r in range(4):
             _, w, b = synthetic.linear_inputs(1, K, N, seed=200 + r)
@@ -432,15 +487,16 @@ def wide_block(torch, dq, synthetic, stream, peaks, reps=24):
             assert l.last_error() == 0, "device-side wait timed out"
         us = statistics.median(t)
         tflops = 2.0 * M * K * N / (us * 1e-6) / 1e12
-        peak = peaks["bf16_tflops"] * (2.0 if fmt == "fp8_static" else 1.0)
+        peak = peaks["bf16_tflops"] * tensor_peak_ratio(fmt)
         out[fmt] = {"us": round(us, 2), "TFLOP/s": round(tflops, 1), "frac_tensor": round(tflops / peak, 4),
                     "peak_tflops": round(peak, 1)}
         del g
         for l in layers:
             l.close()
     out["shape"] = {"M": M, "K": K, "N": N}
-    out["peak_source"] = (f"{peaks['source']} bf16 dense (burst); FP8 = 2x the bf16 figure "
-                          "(the dense FP8:BF16 ratio)")
+    out["peak_source"] = (f"{peaks['source']} bf16 dense (burst); FP8 = 2x and FP4 = 4x the bf16 figure "
+                          "(the dense FP8:BF16 and FP4:BF16 ratios); static FP8 and W4A4 include their "
+                          "activation-quantize kernels")
     return out
 
 
@@ -787,7 +843,7 @@ def run_sweep(args):
                 byts = algorithmic_bytes(fmt, M, K, N, bias=fmt != "fp8_static")
                 gbs = byts / (us * 1e-6) / 1e9
                 tflops = flops / (us * 1e-6) / 1e12
-                peak_t = peaks["bf16_tflops"] * (2.0 if fmt == "fp8_static" else 1.0)
+                peak_t = peaks["bf16_tflops"] * tensor_peak_ratio(fmt)
                 print(json.dumps({"fmt": fmt, "M": M, "K": K, "N": N, "us": round(us, 3),
                                   "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
                                   "TFLOP/s": round(tflops, 1), "frac_tensor": round(tflops / peak_t, 4),
@@ -814,7 +870,8 @@ def main():
     ap.add_argument("--sweep-m", default="1,16,32,128,1024,4096")
     ap.add_argument("--sweep-kn", default="4096x4096,4096x14336,14336x4096")
     ap.add_argument("--sweep-formats", default="int4,nvfp4,mxfp4,fp8,fp8_static")
-    ap.add_argument("--ncu-case", choices=list(LIN_FORMATS) + ["fp8_static", "int4_asym"], default=None,
+    ap.add_argument("--ncu-case", choices=list(LIN_FORMATS) + ["fp8_static", "int4_asym"] + list(W4A4_FORMATS),
+                    default=None,
                     help="small profiling case: 8 plain launches of one format (4 weight sets, no graphs, "
                          "no timing) for an ncu capture; the step's shape unless --ncu-shape is given")
     ap.add_argument("--ncu-shape", default=None, help="MxKxN of the profiling case, e.g. 4096x4096x4096")

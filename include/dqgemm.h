@@ -84,6 +84,17 @@ extern "C" {
  *                  scales [N, K/128] followed by the u8 zero points
  *                  [N, K/128] in [0, 15]; weight = (code - z) * s;
  *                  K % 128 == 0
+ *   DQ_W4A4_MXFP4  FP4 x FP4 ("TorchAO MXFP4 Dynamic Activation + MX Weight
+ *                  (Linear)", intro: MX dynamic activation + MX weight, native
+ *                  MXFP4 x MXFP4 on B200): the weight in DQ_MXFP4 storage;
+ *                  each call quantizes x to MXFP4 (E8M0 per 32 along K, the
+ *                  weight's recipe) and runs the tensor core's block-scaled
+ *                  FP4 MMA, y = sum_k deq(Q(x)) deq(W) + b.
+ *                  K % 32 == 0, N % 32 == 0
+ *   DQ_W4A4_NVFP4  the same with NVFP4: the weight in DQ_NVFP4 storage
+ *                  (global_scale = g_w); x quantized per call with its own
+ *                  global scale g_x = amax(x) / 2688 and E4M3 scales per 16.
+ *                  K % 16 == 0, N % 16 == 0
  */
 typedef enum {
   DQ_INT4_G128 = 0,
@@ -91,7 +102,9 @@ typedef enum {
   DQ_MXFP4 = 2,
   DQ_FP8_WO = 3,
   DQ_FP8_STATIC = 4,
-  DQ_INT4_ASYM_G128 = 5
+  DQ_INT4_ASYM_G128 = 5,
+  DQ_W4A4_MXFP4 = 6,
+  DQ_W4A4_NVFP4 = 7
 } dqgemm_format;
 
 typedef enum {
@@ -119,7 +132,9 @@ typedef struct dqgemm_s* dqgemm_handle;
  * non-negative E4M3), an MXFP4 exponent 0xFF.  An MXFP4 handle whose largest
  * block exponent code emax exceeds 128 needs every block holding a nonzero
  * element to have a code >= emax - 133 (the bf16 operand of the prologue
- * covers a span of 2^133 exactly); DQ_ERR_UNSUPPORTED otherwise. */
+ * covers a span of 2^133 exactly); DQ_ERR_UNSUPPORTED otherwise.  (The W4A4
+ * formats take every non-NaN exponent: their scales go to the tensor core
+ * unchanged.) */
 dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt, int K, int N,
                             const void* packed_w, const void* scales,
                             float global_scale, const void* bias);
@@ -133,7 +148,14 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt, int K, int N,
  * kernel streams its weights before waiting for the previous kernel in the
  * stream, and reads x / writes y only after that wait.  Device-side wait
  * timeouts are reported through dqgemm_last_error after the stream has been
- * synchronized. */
+ * synchronized.
+ * W4A4 handles launch two kernels (MXFP4: quantize x, GEMM) or three (NVFP4:
+ * amax of x, quantize, GEMM), chained the same way.  The quantized x lives
+ * in a workspace the handle owns (dqgemm_plan.workspace_bytes for M): a call
+ * that needs more than the handle holds allocates it, after synchronizing the
+ * device, so make the first call of the largest M before any stream capture.
+ * Calls on one W4A4 handle share that workspace and must be stream-ordered
+ * (not concurrent on different streams). */
 dqgemm_status dqgemm_run(dqgemm_handle h, const void* x, int M, void* y, void* stream);
 
 /* DQ_FP8_STATIC only: the GEMM on activations already quantized by
@@ -203,6 +225,19 @@ dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream);
  * alignment (the one exception to the 16-byte rule above). */
 dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x,
                                       void* q, void* stream);
+
+/* FP4 activation quantization, the first step of a W4A4 call, into the
+ * canonical storage of the weight formats (the same recipe as the packers
+ * below, applied per call to each row of x).  fmt DQ_MXFP4 or DQ_W4A4_MXFP4:
+ * codes u8 [M, K/2] (E2M1 nibbles, low nibble = even k), scales u8 [M, K/32]
+ * E8M0; K % 32 == 0.  fmt DQ_NVFP4 or DQ_W4A4_NVFP4: g_x = amax(x) / 2688
+ * (1 for a zero x) written to the device float *g_x, then scales u8
+ * [M, K/16] E4M3 under g_x and the codes; K % 16 == 0.  x: device bf16
+ * [M, K], 16-byte aligned; codes, scales: device.  The NVFP4 form reduces
+ * the amax in a static device scratch shared by all calls: calls that
+ * overlap on the GPU race.  DQ_ERR_UNSUPPORTED for other formats. */
+dqgemm_status dqgemm_quantize_act_fp4(dqgemm_format fmt, const void* x, int M, int K,
+                                      void* codes, void* scales, float* g_x, void* stream);
 
 /* Quantize and pack a host fp32 weight [N, K] into the canonical layout of
  * `fmt` (host outputs `packed` and `scales`, sized as listed above).  The

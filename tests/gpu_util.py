@@ -36,15 +36,30 @@ def bf16_values(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
+def base_fmt(fmt):
+    """The oracle's storage format of a library format."""
+    return {"fp8_static": "fp8", "w4a4_mxfp4": "mxfp4", "w4a4_nvfp4": "nvfp4"}.get(fmt, fmt)
+
+
 def make_layer(fmt, W, bias_t=None, act_scale=None):
     """Quantize W (fp64 numpy of fp32 values) with the oracle and build a
     handle from that storage.  Returns (handle, storage dict, exact DQ)."""
-    st = L.quantize_pack("fp8" if fmt == "fp8_static" else fmt, W)
+    st = L.quantize_pack(base_fmt(fmt), W)
     g = act_scale if fmt == "fp8_static" else st["global_scale"]
     N, K = W.shape
     h = dq.dqgemm_create(fmt, K, N, dev(st["packed"]), scales_tensor(fmt, st["scales"]), g, bias_t)
-    wdq = L.dequant_exact("fp8" if fmt == "fp8_static" else fmt, st["packed"], st["scales"], st["global_scale"])
+    wdq = L.dequant_exact(base_fmt(fmt), st["packed"], st["scales"], st["global_scale"])
     return h, st, wdq
+
+
+def w4a4_effective_x(fmt, x):
+    """The activation values an FP4 x FP4 layer multiplies: the oracle's
+    dynamic quantization of x (its bf16 values), dequantized exactly."""
+    if fmt == "w4a4_mxfp4":
+        c, s = L.quantize_act_mxfp4(x)
+        return F.e2m1_decode(c) * np.repeat(F.e8m0_decode(s), 32, axis=1)
+    c, s, g = L.quantize_act_nvfp4(x)
+    return F.e2m1_decode(c) * np.repeat(F.e4m3_decode(s), 16, axis=1) * float(g)
 
 
 def run(h, x_t, N):

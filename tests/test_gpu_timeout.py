@@ -17,12 +17,12 @@ import weight_only_quantized_prologue_b200 as dq
 from oracle import linear as L
 from weight_only_quantized_prologue_b200 import synthetic
 
-from gpu_util import bf16_values, check_close, make_layer, static_effective_x
+from gpu_util import base_fmt, bf16_values, check_close, make_layer, static_effective_x, w4a4_effective_x
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "fp8", "fp8_static"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "fp8", "fp8_static", "w4a4_mxfp4", "w4a4_nvfp4"])
 @pytest.mark.parametrize("M,K,N", [(32, 3072, 4096), (1, 1024, 512), (256, 256, 19200)])
 def test_gemm_wait_limit_expires_then_context_recovers(fmt, M, K, N):
     x, w, b = synthetic.linear_inputs(M, K, N, seed=31)
@@ -43,8 +43,13 @@ def test_gemm_wait_limit_expires_then_context_recovers(fmt, M, K, N):
         dq.dqgemm_run(h, xc, M, y)
         torch.cuda.synchronize()
         assert dq.dqgemm_last_error(h) == 0
-        x_eff = static_effective_x(xv, s_x) if fmt == "fp8_static" else xv
-        check_close(bf16_values(y), L.linear_ref(x_eff, wdq, bf16_values(b)), x_eff, wdq)
+        if fmt.startswith("w4a4"):
+            ref = L.w4a4_linear_ref(base_fmt(fmt), xv, st["packed"], st["scales"], st["global_scale"],
+                                    bf16_values(b))
+            check_close(bf16_values(y), ref, w4a4_effective_x(fmt, xv), wdq)
+        else:
+            x_eff = static_effective_x(xv, s_x) if fmt == "fp8_static" else xv
+            check_close(bf16_values(y), L.linear_ref(x_eff, wdq, bf16_values(b)), x_eff, wdq)
     finally:
         dq.dqgemm_destroy(h)
 

@@ -22,6 +22,7 @@ from ._native import (  # noqa: F401
     dqgemm_pack_device,
     dqgemm_pack_device_noalloc,
     dqgemm_pack_host,
+    dqgemm_quantize_act_fp4,
     dqgemm_quantize_act_fp8,
     dqgemm_run,
     dqgemm_run_fp8_static_quantized,

@@ -14,7 +14,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdqgemm.so")
 
-FORMATS = {"int4": 0, "nvfp4": 1, "mxfp4": 2, "fp8": 3, "fp8_static": 4, "int4_asym": 5}
+FORMATS = {"int4": 0, "nvfp4": 1, "mxfp4": 2, "fp8": 3, "fp8_static": 4, "int4_asym": 5,
+           "w4a4_mxfp4": 6, "w4a4_nvfp4": 7}
 STATUS_NAMES = {0: "DQ_OK", 1: "DQ_ERR_INVALID_ARG", 2: "DQ_ERR_UNSUPPORTED", 3: "DQ_ERR_ALIGNMENT",
                 4: "DQ_ERR_ALLOC", 5: "DQ_ERR_CUDA", 6: "DQ_ERR_TIMEOUT"}
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_ALIGNMENT = 0, 1, 2, 3
@@ -48,6 +49,7 @@ _SIGNATURES = {
     "dqgemm_destroy": [_VP],
     "dqgemm_dequantize": [_VP, _VP, _VP],
     "dqgemm_quantize_act_fp8": [_VP, _I, _I, _F, _VP, _VP],
+    "dqgemm_quantize_act_fp4": [_I, _VP, _I, _I, _VP, _VP, _VP, _VP],
     "dqgemm_pack_host": [_I, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_F)],
     "dqgemm_pack_device": [_I, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_F), _VP],
     "dqgemm_pack_device_noalloc": [_I, _VP, _I, _I, _VP, _VP, ctypes.POINTER(_F), _VP],
@@ -105,9 +107,9 @@ def storage_shapes(fmt, K, N):
         return (N, K // 2), np.uint8, (N, K // 128), np.uint16
     if fmt == "int4_asym":   # bf16 scales [N, K/128] then u8 zero points [N, K/128], one buffer
         return (N, K // 2), np.uint8, (3 * N * (K // 128),), np.uint8
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "w4a4_nvfp4"):
         return (N, K // 2), np.uint8, (N, K // 16), np.uint8
-    if fmt == "mxfp4":
+    if fmt in ("mxfp4", "w4a4_mxfp4"):
         return (N, K // 2), np.uint8, (N, K // 32), np.uint8
     return (N, K), np.uint8, (N,), np.float32
 
@@ -159,6 +161,13 @@ def dqgemm_dequantize(h, w_bf16, stream=None):
 def dqgemm_quantize_act_fp8(x, M, K, s_x, q, stream=None):
     _check(lib().dqgemm_quantize_act_fp8(_ptr(x), M, K, float(s_x), _ptr(q), _stream(stream)),
            "dqgemm_quantize_act_fp8")
+
+
+def dqgemm_quantize_act_fp4(fmt, x, M, K, codes, scales, g_x=None, stream=None):
+    """FP4 activation quantization into canonical storage; g_x is a device
+    float32 tensor of one element (NVFP4 formats)."""
+    _check(lib().dqgemm_quantize_act_fp4(FORMATS[fmt], _ptr(x), int(M), int(K), _ptr(codes), _ptr(scales),
+                                         _ptr(g_x), _stream(stream)), "dqgemm_quantize_act_fp4")
 
 
 def dqgemm_pack_host(fmt, W):

@@ -30,6 +30,10 @@ struct dqgemm_s {
   int mx_bias = 126;
   long long weight_bytes = 0;       // canonical packed + scale bytes
   int max_clusters[4][9] = {};      // co-resident clusters per (BN index, cluster size), 0 = unknown
+  // FP4 x FP4: the activation workspace (codes, scale words, the NVFP4 amax
+  // partials, ticket and g_x), grown on demand and reused by every call
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
   unsigned long long timeout_ns = 0;  // limit of the kernels' pipeline waits
   // activation tensor maps already encoded, by (x, M, tile rows, e4m3 input):
   // encoding one costs host time on every call, and layers see the same
@@ -70,8 +74,15 @@ bool is_device_ptr(const void* p) {
 }
 
 // canonical storage sizes of dqgemm.h
-size_t packed_bytes(int fmt, int K, int N) { return is_4bit(fmt) ? (size_t)N * K / 2 : (size_t)N * K; }
+// the canonical storage of a W4A4 handle is that of its weight format
+int storage_fmt(int fmt) { return fmt == FMT_W4A4MX ? FMT_MXFP4 : fmt == FMT_W4A4NV ? FMT_NVFP4 : fmt; }
+
+size_t packed_bytes(int fmt, int K, int N) {
+  fmt = storage_fmt(fmt);
+  return is_4bit(fmt) ? (size_t)N * K / 2 : (size_t)N * K;
+}
 size_t scale_bytes(int fmt, int K, int N) {
+  fmt = storage_fmt(fmt);
   switch (fmt) {
     case FMT_INT4: return (size_t)N * (K / 128) * 2;
     case FMT_INT4A: return (size_t)N * (K / 128) * 3;   // bf16 scales, then u8 zero points
@@ -82,8 +93,8 @@ size_t scale_bytes(int fmt, int K, int N) {
 }
 
 dqgemm_status check_shape(int fmt, int K, int N) {
-  if (fmt < 0 || fmt > FMT_INT4A || K <= 0 || N <= 0) return DQ_ERR_INVALID_ARG;
-  switch (fmt) {
+  if (fmt < 0 || fmt > FMT_W4A4NV || K <= 0 || N <= 0) return DQ_ERR_INVALID_ARG;
+  switch (storage_fmt(fmt)) {
     case FMT_INT4:
     case FMT_INT4A: return K % 128 ? DQ_ERR_INVALID_ARG : DQ_OK;
     case FMT_NVFP4: return (K % 16 || N % 16) ? DQ_ERR_INVALID_ARG : DQ_OK;
@@ -113,7 +124,24 @@ void relayout(int fmt, int K, int N, int KS, int NT, const std::vector<uint8_t>&
       uint8_t* ch = out.data() + ((size_t)t * KS + s) * CH;
       for (int r = 0; r < TILE_N; ++r) {
         const int n = t * TILE_N + r;
-        if (is_4bit(fmt)) {
+        if (is_w4a4(fmt)) {
+          // swizzled K-major image of the packed codes (256 k = 128 bytes a
+          // row), then the scale words [k-step t4][row]
+          for (int b = 0; b < 128; ++b) {
+            const int k = s * W4_STAGE_K + 2 * b;
+            ch[r * 128 + (((b >> 4) ^ (r & 7)) << 4) + (b & 15)] = (uint8_t)(nib(n, k) | (nib(n, k + 1) << 4));
+          }
+          const bool mx = fmt == FMT_W4A4MX;
+          const int vs = mx ? 32 : 16, blocks = K / vs, per_step = 64 / vs;
+          for (int t4 = 0; t4 < 4; ++t4) {
+            uint32_t word = 0;
+            for (int j = 0; j < per_step; ++j) {
+              const int blk = (s * W4_STAGE_K + t4 * 64) / vs + j;
+              if (n < N && blk < blocks) word |= (uint32_t)scales[(size_t)n * blocks + blk] << (8 * j);
+            }
+            put32(ch + W4_SF_OFF + (t4 * TILE_N + r) * 4, word);
+          }
+        } else if (is_4bit(fmt)) {
           for (int h = 0; h < 2; ++h)
             for (int j = 0; j < 2; ++j)
               for (int w = 0; w < 4; ++w) {
@@ -248,7 +276,7 @@ struct GemmLauncher {
   using C = GemmCfg<FMT, BN>;
   static cudaError_t set_attr() {
     cudaError_t e = set_attr_q<false>();
-    if constexpr (FMT != FMT_MLP) {
+    if constexpr (FMT != FMT_MLP && !is_w4a4(FMT)) {
       if (e == cudaSuccess) e = set_attr_q<true>();
     }
     return e;
@@ -290,7 +318,7 @@ struct GemmLauncher {
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attrs[2];
     config(cfg, attrs, grid, p.split, st);
-    if constexpr (FMT == FMT_MLP) {
+    if constexpr (FMT == FMT_MLP || is_w4a4(FMT)) {
       return cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, false>, tm, p);
     } else {
       return p.yq ? cudaLaunchKernelEx(&cfg, dq_gemm_kernel<FMT, BN, true>, tm, p)
@@ -315,7 +343,7 @@ struct GemmLauncher {
 template <int FMT>
 int stages_for(int bn) {
   switch (bn) {
-    case 16: return GemmCfg<FMT, 16>::STAGES;
+    case 16: return GemmCfg<FMT, is_w4a4(FMT) ? 32 : 16>::STAGES;
     case 32: return GemmCfg<FMT, 32>::STAGES;
     case 64: return GemmCfg<FMT, 64>::STAGES;
     case 128: return GemmCfg<FMT, 128>::STAGES;
@@ -327,7 +355,7 @@ int stages_for(int bn) {
 template <int FMT>
 int xstages_for(int bn) {
   switch (bn) {
-    case 16: return GemmCfg<FMT, 16>::XST;
+    case 16: return GemmCfg<FMT, is_w4a4(FMT) ? 32 : 16>::XST;
     case 32: return GemmCfg<FMT, 32>::XST;
     case 64: return GemmCfg<FMT, 64>::XST;
     case 128: return GemmCfg<FMT, 128>::XST;
@@ -339,7 +367,7 @@ int xstages_for(int bn) {
 template <int FMT>
 int smem_for(int bn) {
   switch (bn) {
-    case 16: return GemmCfg<FMT, 16>::SMEM;
+    case 16: return GemmCfg<FMT, is_w4a4(FMT) ? 32 : 16>::SMEM;
     case 32: return GemmCfg<FMT, 32>::SMEM;
     case 64: return GemmCfg<FMT, 64>::SMEM;
     case 128: return GemmCfg<FMT, 128>::SMEM;
@@ -350,7 +378,8 @@ int smem_for(int bn) {
 }
 template <int FMT>
 cudaError_t set_attrs() {
-  cudaError_t e = GemmLauncher<FMT, 16>::set_attr();
+  // (W4A4 x tiles hold 32 rows or more: there is no 16-row instance)
+  cudaError_t e = GemmLauncher<FMT, is_w4a4(FMT) ? 32 : 16>::set_attr();
   if (e == cudaSuccess) e = GemmLauncher<FMT, 32>::set_attr();
   if (e == cudaSuccess) e = GemmLauncher<FMT, 64>::set_attr();
   if (e == cudaSuccess) e = GemmLauncher<FMT, 128>::set_attr();
@@ -362,7 +391,9 @@ cudaError_t set_attrs() {
 template <int FMT>
 cudaError_t launch_fmt(int bn, const CUtensorMap& tm, const GemmParams& p, int grid, cudaStream_t st) {
   switch (bn) {
-    case 16: return GemmLauncher<FMT, 16>::launch(tm, p, grid, st);
+    case 16:
+      if constexpr (is_w4a4(FMT)) return cudaErrorInvalidValue;   // never planned
+      else return GemmLauncher<FMT, 16>::launch(tm, p, grid, st);
     case 32: return GemmLauncher<FMT, 32>::launch(tm, p, grid, st);
     case 64: return GemmLauncher<FMT, 64>::launch(tm, p, grid, st);
     case 128: return GemmLauncher<FMT, 128>::launch(tm, p, grid, st);
@@ -375,7 +406,7 @@ cudaError_t launch_fmt(int bn, const CUtensorMap& tm, const GemmParams& p, int g
 template <int FMT>
 int max_clusters_fmt(int bn, int split) {
   switch (bn) {
-    case 16: return GemmLauncher<FMT, 16>::max_active_clusters(split);
+    case 16: return GemmLauncher<FMT, is_w4a4(FMT) ? 32 : 16>::max_active_clusters(split);
     case 32: return GemmLauncher<FMT, 32>::max_active_clusters(split);
     case 64: return GemmLauncher<FMT, 64>::max_active_clusters(split);
     default: return GemmLauncher<FMT, 128>::max_active_clusters(split);
@@ -389,6 +420,8 @@ int max_clusters_fmt(int bn, int split) {
     case FMT_NVFP4: { constexpr int F = FMT_NVFP4; CALL; } break; \
     case FMT_MXFP4: { constexpr int F = FMT_MXFP4; CALL; } break; \
     case FMT_FP8: { constexpr int F = FMT_FP8; CALL; } break;     \
+    case FMT_W4A4MX: { constexpr int F = FMT_W4A4MX; CALL; } break; \
+    case FMT_W4A4NV: { constexpr int F = FMT_W4A4NV; CALL; } break; \
     default: { constexpr int F = FMT_FP8S; CALL; } break;         \
   }
 
@@ -417,6 +450,7 @@ int cluster_capacity(dqgemm_s* h, int bn, int split) {
 // its MMA time).  The fused static-FP8 kernel stays at 128 rows.
 int pick_bn(const dqgemm_s* h, int M, bool xq) {
   int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  if (is_w4a4(h->fmt) && bn < 32) bn = 32;   // one block-scale column per 32 x rows
   if (M > 128 && !(h->fmt == FMT_FP8S && !xq)) {
     const long long sms = h->num_sms, nt = h->n_tiles;
     const long long t256 = (M + 255) / 256 * nt, t128 = (M + 127) / 128 * nt;
@@ -425,6 +459,25 @@ int pick_bn(const dqgemm_s* h, int M, bool xq) {
   }
   return bn;
 }
+
+// The FP4 x FP4 activation workspace for M rows in x tiles of bn rows: the
+// NVFP4 amax partials, the amax ticket and g_x at fixed offsets (the ticket
+// is zeroed once, when the workspace is allocated, and left at zero by every
+// call), then codes [rows][kp / 2] and scale words [m_tiles][k_stages][4][bn].
+struct W4Workspace {
+  static constexpr size_t partials = 0, ticket = (size_t)kActAmaxBlocks * 4, gx = ticket + 16, codes = 8192;
+  int rows = 0, kp = 0;
+  size_t sfw = 0, total = 0;
+};
+W4Workspace w4a4_workspace(const dqgemm_s* h, int M, int bn) {
+  W4Workspace w;
+  w.rows = (M + bn - 1) / bn * bn;
+  w.kp = h->k_stages * W4_STAGE_K;
+  w.sfw = W4Workspace::codes + (size_t)w.rows * (w.kp / 2);
+  w.total = w.sfw + (size_t)w.rows * h->k_stages * 16;
+  return w;
+}
+static_assert(W4Workspace::gx + 16 <= W4Workspace::codes, "workspace header");
 
 void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl, bool xq = false) {
   std::memset(pl, 0, sizeof(*pl));
@@ -472,7 +525,7 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl, bool xq = false) {
   }
   pl->stages = st;
   pl->smem_bytes = sm;
-  pl->workspace_bytes = 0;
+  pl->workspace_bytes = is_w4a4(h->fmt) ? (long long)w4a4_workspace(h, M, bn).total : 0;
   pl->weight_bytes = h->weight_bytes;
   pl->x_stages = xs;
   // the split gives rank q the stages [q*KS/S, (q+1)*KS/S); whole tiles give
@@ -484,7 +537,7 @@ void fill_plan(dqgemm_s* h, int M, dqgemm_plan* pl, bool xq = false) {
 // The activation tensor map for (x, M, tile rows, e4m3 input), from the
 // handle's cache or freshly encoded.  A map encodes only those and K, so a
 // cached one for the same key is the map this call would encode.
-bool x_map(dqgemm_s* h, const void* x, int M, int bn, bool xq, CUtensorMap* tm, bool* x3d) {
+bool x_map(dqgemm_s* h, const void* x, int M, int bn, bool xq, CUtensorMap* tm, bool* x3d, int q_row_bytes = 0) {
   std::lock_guard<std::mutex> lock(h->maps_mu);
   for (const auto& e : h->maps) {
     if (e.x == x && e.M == M && e.bn == bn && e.xq == xq) {
@@ -493,7 +546,8 @@ bool x_map(dqgemm_s* h, const void* x, int M, int bn, bool xq, CUtensorMap* tm, 
       return true;
     }
   }
-  if (xq ? !make_q_map(tm, x, M, h->K, bn) : !make_x_map(tm, x, M, h->K, bn, x3d)) return false;
+  if (xq ? !make_q_map(tm, x, M, q_row_bytes ? q_row_bytes : h->K, bn) : !make_x_map(tm, x, M, h->K, bn, x3d))
+    return false;
   auto& e = h->maps[h->next_map];
   h->next_map = (h->next_map + 1) % dqgemm_s::kMaps;
   e.x = x;
@@ -506,6 +560,30 @@ bool x_map(dqgemm_s* h, const void* x, int M, int bn, bool xq, CUtensorMap* tm, 
 }
 
 dqgemm_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA; }
+
+// a small kernel in the programmatic-dependent-launch chain of the GEMMs
+// (its first instruction waits for the previous grid)
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kern)(KArgs...), int grid, int block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.stream = st;
+  cudaLaunchAttribute a[1];
+  int na = 0;
+  if (pdl_enabled()) {
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = 1;
+    na = 1;
+  }
+  cfg.attrs = a;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+int act_amax_grid(long long count) {
+  return (int)std::max<long long>(1, std::min<long long>((count / 8 + 255) / 256, kActAmaxBlocks));
+}
 
 // Codes the canonical storage may hold (the packers produce nothing else):
 //   FP8 formats  no NaN weight code (0x7F / 0xFF)
@@ -521,9 +599,13 @@ dqgemm_status check_codes(int fmt, int K, int N, const std::vector<uint8_t>& hp,
   if (fmt == FMT_FP8 || fmt == FMT_FP8S) {
     for (uint8_t c : hp)
       if ((c & 0x7F) == 0x7F) return DQ_ERR_INVALID_ARG;
-  } else if (fmt == FMT_NVFP4) {
+  } else if (fmt == FMT_NVFP4 || fmt == FMT_W4A4NV) {
     for (uint8_t c : hs)
       if (c >= 0x7F) return DQ_ERR_INVALID_ARG;
+  } else if (fmt == FMT_W4A4MX) {
+    // the tensor core takes every E8M0 exponent but the NaN code
+    for (uint8_t c : hs)
+      if (c == 255) return DQ_ERR_INVALID_ARG;
   } else if (fmt == FMT_MXFP4) {
     int cmax = 0;
     for (uint8_t c : hs) {
@@ -568,6 +650,7 @@ dqgemm_status dqgemm_destroy(dqgemm_handle h) {
   if (!h) return DQ_ERR_INVALID_ARG;
   cudaDeviceSynchronize();
   cudaFree(h->wchunks);
+  cudaFree(h->ws);
   cudaFree(h->col_scale);
   cudaFree(h->bias);
   if (h->status_host) cudaFreeHost(h->status_host);
@@ -586,7 +669,7 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   if (!aligned16(packed_w) || !aligned16(scales) || (bias && !aligned16(bias))) return DQ_ERR_ALIGNMENT;
   if (!is_device_ptr(packed_w) || !is_device_ptr(scales) || (bias && !is_device_ptr(bias)))
     return DQ_ERR_INVALID_ARG;
-  if ((fmt == FMT_NVFP4 || fmt == FMT_FP8S) && !(std::isfinite(global_scale) && global_scale > 0.f))
+  if ((fmt == FMT_NVFP4 || fmt == FMT_W4A4NV || fmt == FMT_FP8S) && !(std::isfinite(global_scale) && global_scale > 0.f))
     return DQ_ERR_INVALID_ARG;
 
   std::vector<uint8_t> hp(packed_bytes(fmt, K, N)), hs(scale_bytes(fmt, K, N));
@@ -600,7 +683,8 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   h->fmt = fmt;
   h->K = K;
   h->N = N;
-  h->k_stages = (K + STAGE_K - 1) / STAGE_K;
+  const int stage_k = is_w4a4(fmt) ? W4_STAGE_K : STAGE_K;
+  h->k_stages = (K + stage_k - 1) / stage_k;
   h->n_tiles = (N + TILE_N - 1) / TILE_N;
   h->weight_bytes = (long long)(hp.size() + hs.size());
   h->timeout_ns = timeout_ns();
@@ -619,6 +703,8 @@ dqgemm_status dqgemm_create(dqgemm_handle* out, dqgemm_format fmt_, int K, int N
   } else if (fmt == FMT_FP8S) {
     h->sigma = global_scale;
     h->s_x = global_scale;
+  } else if (fmt == FMT_W4A4NV) {
+    h->sigma = global_scale;           // g_w; the call's g_x is applied on the device
   }
 
   std::vector<uint8_t> chunks;
@@ -662,9 +748,85 @@ dqgemm_status dqgemm_get_plan(dqgemm_handle h, int M, dqgemm_plan* plan) {
   return DQ_OK;
 }
 
+// FP4 x FP4: quantize x into the handle's workspace (NVFP4: its amax first),
+// then the block-scaled GEMM on those codes; three or two launches chained by
+// programmatic dependent launch.
+static dqgemm_status run_w4a4(dqgemm_handle h, const void* x, int M, void* y, void* stream) {
+  dqgemm_plan pl;
+  fill_plan(h, M, &pl);
+  const W4Workspace w = w4a4_workspace(h, M, pl.bn);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  {
+    std::lock_guard<std::mutex> lock(h->maps_mu);
+    if (h->ws_bytes < w.total) {
+      // grow: calls already launched may still read the old workspace
+      cudaError_t e = cudaDeviceSynchronize();
+      cudaFree(h->ws);
+      h->ws = nullptr;
+      h->ws_bytes = 0;
+      if (e != cudaSuccess) return DQ_ERR_CUDA;
+      if (cudaMalloc(&h->ws, w.total) != cudaSuccess) {
+        h->ws = nullptr;
+        return DQ_ERR_ALLOC;
+      }
+      if (cudaMemset(h->ws, 0, w.total) != cudaSuccess) return DQ_ERR_CUDA;
+      h->ws_bytes = w.total;
+    }
+  }
+  uint8_t* codes = h->ws + W4Workspace::codes;
+  uint32_t* sfw = reinterpret_cast<uint32_t*>(h->ws + w.sfw);
+  float* gx = reinterpret_cast<float*>(h->ws + W4Workspace::gx);
+  const bool mx = h->fmt == FMT_W4A4MX;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  cudaError_t e = cudaSuccess;
+  if (!mx) {
+    const long long count = (long long)M * h->K;
+    e = launch_chained(act_amax_kernel, act_amax_grid(count), 256, s, xb, count,
+                       reinterpret_cast<float*>(h->ws + W4Workspace::partials),
+                       reinterpret_cast<unsigned int*>(h->ws + W4Workspace::ticket), gx);
+  }
+  if (e == cudaSuccess) {
+    const long long threads = (long long)w.rows * (w.kp / 64);
+    const int grid = (int)std::min<long long>((threads + 255) / 256, 148 * 8);
+    e = mx ? launch_chained(w4a4_act_quant_kernel<true>, grid, 256, s, xb, M, h->K, w.rows, w.kp, pl.bn,
+                            (const float*)gx, codes, sfw, (uint8_t*)nullptr)
+           : launch_chained(w4a4_act_quant_kernel<false>, grid, 256, s, xb, M, h->K, w.rows, w.kp, pl.bn,
+                            (const float*)gx, codes, sfw, (uint8_t*)nullptr);
+  }
+  if (e != cudaSuccess) return DQ_ERR_CUDA;
+  CUtensorMap tm;
+  bool x3d = false;
+  if (!x_map(h, codes, w.rows, pl.bn, true, &tm, &x3d, w.kp / 2)) return DQ_ERR_CUDA;
+  GemmParams p{};
+  p.wchunks = h->wchunks;
+  p.bias = h->bias;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.status = h->status;
+  p.sigma = h->sigma;
+  p.s_x = 1.f;
+  p.s_out = 1.f;
+  p.M = M;
+  p.N = h->N;
+  p.k_stages = h->k_stages;
+  p.m_tiles = pl.m_tiles;
+  p.tiles = pl.m_tiles * pl.n_tiles;
+  p.split = pl.max_segments;
+  p.timeout_ns = h->timeout_ns;
+  p.drain_ns = std::max(timeout_ns(), kDefaultTimeoutNs);
+  p.xsf = sfw;
+  p.gx = mx ? nullptr : gx;
+  DQ_FMT_SWITCH(h->fmt, e = launch_fmt<F>(pl.bn, tm, p, pl.grid, s));
+  return cuda_err(e);
+}
+
 static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, void* y, bool yq, float s_out,
                               void* stream) {
   if (!h || !x || !y || M < 1) return DQ_ERR_INVALID_ARG;
+  if (is_w4a4(h->fmt)) {
+    if (xq || yq) return DQ_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
+    return run_w4a4(h, x, M, y, stream);
+  }
   if (yq && !(std::isfinite(s_out) && s_out > 0.f)) return DQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return DQ_ERR_ALIGNMENT;
   dqgemm_plan pl;
@@ -772,15 +934,24 @@ dqgemm_status dqgemm_run_static_mlp(dqgemm_handle l1, dqgemm_handle l2, const vo
   return cuda_err(e);
 }
 
+extern "C++" {
+template <int FMT>
+void launch_dequant(const dqgemm_s* h, float sigma, __nv_bfloat16* o, cudaStream_t s) {
+  if constexpr (!is_w4a4(FMT)) {
+    const dim3 grid(h->n_tiles, h->k_stages);
+    dequant_kernel<FMT><<<grid, 256, 0, s>>>(h->wchunks, h->col_scale, sigma, h->mx_bias, h->N, h->K, h->k_stages, o);
+  }
+}
+}
+
 dqgemm_status dqgemm_dequantize(dqgemm_handle h, void* w_bf16, void* stream) {
   if (!h || !w_bf16) return DQ_ERR_INVALID_ARG;
+  if (is_w4a4(h->fmt)) return DQ_ERR_UNSUPPORTED;   // no bf16 operand: the tensor core reads the codes
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dim3 grid(h->n_tiles, h->k_stages);
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(w_bf16);
   // static FP8: the weight alone is e4m3 * s_w[n] (sigma there is the activation scale)
   const float sigma = h->fmt == FMT_FP8S ? 1.f : h->sigma;
-  DQ_FMT_SWITCH(h->fmt, (dequant_kernel<F><<<grid, 256, 0, s>>>(h->wchunks, h->col_scale, sigma, h->mx_bias,
-                                                                 h->N, h->K, h->k_stages, o)));
+  DQ_FMT_SWITCH(h->fmt, launch_dequant<F>(h, sigma, o, s));
   return cuda_err(cudaGetLastError());
 }
 
@@ -810,9 +981,50 @@ dqgemm_status dqgemm_quantize_act_fp8(const void* x, int M, int K, float s_x, vo
   return cuda_err(cudaGetLastError());
 }
 
+namespace {
+// the canonical FP4 activation quantizer's NVFP4 amax scratch: partial
+// maxima, then the ticket (zero-initialized, left at zero by every call)
+static __device__ __align__(256) float g_act_fp4_scratch[kActAmaxBlocks + 4];
+}  // namespace
+
+dqgemm_status dqgemm_quantize_act_fp4(dqgemm_format fmt_, const void* x, int M, int K, void* codes, void* scales,
+                                      float* g_x, void* stream) {
+  const int fmt = storage_fmt((int)fmt_);
+  if (fmt != FMT_MXFP4 && fmt != FMT_NVFP4) return DQ_ERR_UNSUPPORTED;
+  const bool mx = fmt == FMT_MXFP4;
+  if (!x || !codes || !scales || M < 1 || K < 1 || K % (mx ? 32 : 16) || (!mx && !g_x)) return DQ_ERR_INVALID_ARG;
+  if (!aligned16(x)) return DQ_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  cudaError_t e = cudaSuccess;
+  if (!mx) {
+    void* scratch = nullptr;
+    if (cudaGetSymbolAddress(&scratch, g_act_fp4_scratch) != cudaSuccess || !scratch) {
+      cudaGetLastError();
+      return DQ_ERR_CUDA;
+    }
+    float* partials = static_cast<float*>(scratch);
+    const long long count = (long long)M * K;
+    e = launch_chained(act_amax_kernel, act_amax_grid(count), 256, s, xb, count, partials,
+                       reinterpret_cast<unsigned int*>(partials + kActAmaxBlocks), g_x);
+  }
+  if (e == cudaSuccess) {
+    const int kp = (K + 63) / 64 * 64;
+    const long long threads = (long long)M * (kp / 64);
+    const int grid = (int)std::min<long long>((threads + 255) / 256, 148 * 8);
+    uint8_t* c = static_cast<uint8_t*>(codes);
+    uint8_t* sc = static_cast<uint8_t*>(scales);
+    e = mx ? launch_chained(w4a4_act_quant_kernel<true>, grid, 256, s, xb, M, K, M, kp, 1, (const float*)g_x, c,
+                            (uint32_t*)nullptr, sc)
+           : launch_chained(w4a4_act_quant_kernel<false>, grid, 256, s, xb, M, K, M, kp, 1, (const float*)g_x, c,
+                            (uint32_t*)nullptr, sc);
+  }
+  return cuda_err(e);
+}
+
 dqgemm_status dqgemm_pack_host(dqgemm_format fmt_, const float* W, int K, int N, void* packed, void* scales,
                                float* global_scale) {
-  const int fmt = (int)fmt_;
+  const int fmt = storage_fmt((int)fmt_);
   dqgemm_status st = check_shape(fmt, K, N);
   if (st != DQ_OK) return st;
   if (!W || !packed || !scales) return DQ_ERR_INVALID_ARG;
@@ -873,7 +1085,7 @@ dqgemm_status dqgemm_pack_host(dqgemm_format fmt_, const float* W, int K, int N,
 
 dqgemm_status dqgemm_pack_device(dqgemm_format fmt_, const float* W, int K, int N, void* packed, void* scales,
                                  float* global_scale, void* stream) {
-  const int fmt = (int)fmt_;
+  const int fmt = storage_fmt((int)fmt_);
   dqgemm_status st = check_shape(fmt, K, N);
   if (st != DQ_OK) return st;
   if (!W || !packed || !scales) return DQ_ERR_INVALID_ARG;
@@ -944,7 +1156,7 @@ float* noalloc_scratch(dqgemm_status* st) {
 
 dqgemm_status dqgemm_pack_device_noalloc(dqgemm_format fmt_, const float* W, int K, int N, void* packed,
                                          void* scales, float* global_scale, void* stream) {
-  const int fmt = (int)fmt_;
+  const int fmt = storage_fmt((int)fmt_);
   dqgemm_status st = check_shape(fmt, K, N);
   if (st != DQ_OK) return st;
   if (!W || !packed || !scales) return DQ_ERR_INVALID_ARG;

@@ -193,6 +193,174 @@ __global__ void amax_final_kernel(const float* partials, int n, unsigned int* am
 }
 
 // ---------------------------------------------------------------------------
+// FP4 x FP4: dynamic activation quantization ("TorchAO MXFP4 Dynamic
+// Activation + MX Weight (Linear)", intro: MX-quantized activations and
+// weights for the native FP4 MMA).  One thread per (row, 64 k): the two MX
+// blocks (E8M0 per 32) or the four NVFP4 blocks (E4M3 per 16, under the
+// call's global scale g_x) of those 64 k, quantized with the weight packer's
+// codec, so that activations and weights follow the same recipe.
+// GEMM layout (sfw set): codes [rows][kp / 2], the even k in the low nibble,
+// rows >= M and k >= K zero; scale words [m_tile][k_stage][t][bn] (k-stage
+// of 256, k-step t of 64; the word layout of the weight chunks).
+// Canonical layout (sfw null): codes [M][K / 2], scale bytes [M][K / VS].
+// ---------------------------------------------------------------------------
+// E2M1 codes of two magnitudes, a at k (low nibble) and b at k + 1: the
+// hardware conversion, round to nearest even, saturating at 6
+__device__ __forceinline__ uint32_t e2m1x2_mag(float a, float b) {
+  uint16_t r;
+  asm("{ .reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "mov.b16 %0, {t, 0};\n\t}"
+      : "=h"(r)
+      : "f"(a), "f"(b));
+  return r;
+}
+
+// The codes of one word of two bf16 values (low half at k): each value
+// times `mul` (MXFP4: the block's 2^-e, a product exact in fp32) or divided
+// by `div` (NVFP4: the block's dec(sb) * g, IEEE division), rounded to E2M1,
+// the sign bit of the input kept (so -0 gives code 8, as the packer's codec
+// does).  Returns the byte of the two codes.
+template <bool MX>
+__device__ __forceinline__ uint32_t e2m1_pair(uint32_t w, float f) {
+  const float lo = __uint_as_float((w & 0x7FFFu) << 16), hi = __uint_as_float(w & 0x7FFF0000u);
+  const uint32_t mag = MX ? e2m1x2_mag(__fmul_rn(lo, f), __fmul_rn(hi, f))
+                          : e2m1x2_mag(__fdiv_rn(lo, f), __fdiv_rn(hi, f));
+  return mag | ((w >> 12) & 0x8u) | ((w >> 24) & 0x80u);
+}
+
+template <bool MX>
+__global__ void __launch_bounds__(256) w4a4_act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
+                                                             int rows, int kp, int bn, const float* gx,
+                                                             uint8_t* codes, uint32_t* sfw, uint8_t* scales) {
+  pdl_wait();   // x may be the previous grid's output, and that grid may still read the workspace
+  pdl_launch_dependents();
+  constexpr int VS = MX ? 32 : 16;   // elements per block
+  constexpr int WB = VS / 2;         // bf16x2 words per block
+  const float g = MX ? 1.f : *reinterpret_cast<const volatile float*>(gx);
+  const int slices = kp / 64;
+  const long long total = (long long)rows * slices;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int row = (int)(i / slices), sl = (int)(i - (long long)row * slices);
+    const int k0 = sl * 64;
+    uint32_t packed[8];
+    uint32_t word = 0;
+#pragma unroll
+    for (int b = 0; b < 64 / VS; ++b) {
+      const int kb = k0 + b * VS;
+      uint32_t w[WB];
+      if (row < M && kb + VS <= K) {
+        // (K is a multiple of 16 and x 16-byte aligned: whole vectors)
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * K + kb);
+#pragma unroll
+        for (int q = 0; q < WB / 4; ++q) {
+          const uint4 u = src[q];
+          w[4 * q] = u.x;
+          w[4 * q + 1] = u.y;
+          w[4 * q + 2] = u.z;
+          w[4 * q + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < WB; ++e) w[e] = 0u;
+      }
+      // block amax: the largest bf16 magnitude (as bits; x holds no NaN)
+      uint32_t am = 0;
+#pragma unroll
+      for (int e = 0; e < WB; ++e) am = max(am, max(w[e] & 0x7FFFu, (w[e] >> 16) & 0x7FFFu));
+      const float amax = __uint_as_float(am << 16);
+      uint32_t sc = 0;
+      float f = 0.f;
+      bool live = amax > 0.f;
+      if constexpr (MX) {
+        if (live) {
+          int e = ilog2f(amax) - 2;
+          e = e < -127 ? -127 : e;   // (amax < 2^128: e <= 125, and 2^-e is an fp32 normal)
+          sc = (uint32_t)(e + 127);
+          f = pow2f(-e);
+        }
+      } else {
+        sc = e4m3_encode_sat(fdiv(fdiv(amax, 6.f), g));
+        f = fmul(e4m3_decode((uint8_t)sc), g);
+        live = f > 0.f;
+      }
+      word |= sc << (8 * b);
+#pragma unroll
+      for (int q = 0; q < WB / 4; ++q) {
+        uint32_t pk = 0;
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk |= e2m1_pair<MX>(w[4 * q + e], f) << (8 * e);
+        }
+        packed[b * (WB / 4) + q] = pk;
+      }
+      if (!sfw && row < M && kb < K) scales[(size_t)row * (K / VS) + kb / VS] = (uint8_t)sc;
+    }
+    if (sfw) {
+      uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)row * (kp / 2) + k0 / 2);
+      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      const int mt = row / bn, r = row - mt * bn, ks = k0 >> 8, t = (k0 >> 6) & 3;
+      sfw[(((size_t)mt * (kp >> 8) + ks) * 4 + t) * bn + r] = word;
+    } else if (row < M) {
+      for (int b = 0; b < 32 && k0 + 2 * b < K; ++b)
+        codes[(size_t)row * (K / 2) + k0 / 2 + b] = (uint8_t)(packed[b >> 2] >> (8 * (b & 3)));
+    }
+  }
+}
+
+// NVFP4 activations: g_x = amax(x) / 2688 (1 for an all-zero x), written to
+// *gx by the last block to finish (the blocks leave their maxima in
+// partials[]; `ticket` counts them and is reset to 0 for the next call).
+constexpr int kActAmaxBlocks = 1024;
+__global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ x, long long count,
+                                                       float* partials, unsigned int* ticket, float* gx) {
+  pdl_wait();
+  pdl_launch_dependents();
+  float a = 0.f;
+  const long long vecs = count / 8;
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < vecs;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint4 u = xv[i];
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      a = fmaxf(a, fmaxf(fabsf(__uint_as_float(w4[e] << 16)), fabsf(__uint_as_float(w4[e] & 0xFFFF0000u))));
+  }
+  for (long long i = vecs * 8 + blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x)
+    a = fmaxf(a, fabsf(__bfloat162float(x[i])));
+  __shared__ float wmax[8];
+  __shared__ int last;
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) a = fmaxf(a, wmax[w]);
+    partials[blockIdx.x] = a;
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == gridDim.x - 1 ? 1 : 0;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  float m = 0.f;
+  for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x)
+    m = fmaxf(m, *reinterpret_cast<const volatile float*>(partials + i));
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+    *gx = nvfp4_global_scale(m);
+    *ticket = 0u;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // bounded-wait self test: waits on a barrier nothing will ever arrive at
 // ---------------------------------------------------------------------------
 __global__ void selftest_timeout_kernel(int* status, unsigned long long timeout_ns) {

@@ -313,6 +313,42 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int bn) {
          | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(TILE_N >> 4) << 24);
 }
 
+// Block-scaled FP4 x FP4 (kind::mxf4 for MXFP4, kind::mxf4nvf4 for NVFP4):
+// A and B packed E2M1 (two codes a byte, the even k in the low nibble),
+// K-major, D fp32, 64 k per MMA.  Bits: 7-9 / 10-12 A / B format (1 = E2M1),
+// 17-22 N / 8, 23 scale format (1 = E8M0, 0 = E4M3), 24-28 M / 16; the scale
+// factors' byte selectors (bits 4-5, 29-30) stay 0: each operand's scale
+// words start at byte 0 of their tensor-memory columns.
+__host__ __device__ constexpr uint32_t idesc_fp4(int bn, bool e8m0) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(bn >> 3) << 17) | ((e8m0 ? 1u : 0u) << 23) |
+         ((uint32_t)(TILE_N >> 4) << 24);
+}
+
+// D (+)= A . B^T with per-block scale factors read from tensor memory: for
+// row m of A the word at lane m % 32 (every lane quadrant holds a copy),
+// column sfa + m / 32, byte j = the scale of the j-th block of this MMA's
+// 64 k (2 blocks of 32 for MXFP4, 4 of 16 for NVFP4); likewise for the rows
+// of B at sfb.
+template <bool MX>
+__device__ __forceinline__ void mma_fp4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  if constexpr (MX) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+  }
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row groups 1024 bytes apart.  `saddr` must lie in a
 // 1024-byte-aligned swizzle atom (plus the k offset within its row).
@@ -328,6 +364,25 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
       "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
+}
+// n consecutive 32-bit columns of this warp's 32 lanes (n = 1, 2, 4, 8)
+template <int NC>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* v) {
+  if constexpr (NC == 1) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v[0]) : "memory");
+  } else if constexpr (NC == 2) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(v[0]), "r"(v[1])
+                 : "memory");
+  } else if constexpr (NC == 4) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3])
+                 : "memory");
+  } else {
+    static_assert(NC == 8, "1, 2, 4 or 8 columns");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+  }
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -66,6 +66,11 @@ struct GemmParams {
   const __nv_bfloat16* bias2;
   __nv_bfloat16* h_out;          // optional: layer 1's bf16 output [M, N]
   int N2;
+  // FP4 x FP4: the activation's block-scale words, [m_tile][k_stage][4][BN]
+  // (the layout of the weight's, per tile of BN rows), and for NVFP4 the
+  // activation's per-call global scale (device, written by the quantizer)
+  const uint32_t* xsf;
+  const float* gx;
 };
 
 // the e4m3 code of an output for the next static-FP8 layer,
@@ -82,20 +87,29 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 
 template <int FMT, int BN>
 struct GemmCfg {
-  // static FP8 with x quantized beforehand: x arrives as e4m3 [M, K] through
-  // a 2-D u8 map (box 128 k x BN rows), straight into the operand buffer
-  static constexpr bool XQ = (FMT == FMT_FP8SQ);
+  // FP4 x FP4 (W4A4): both operands packed E2M1 in shared memory, x
+  // quantized beforehand (codes through a 2-D u8 map, its block-scale words
+  // by a 1-D bulk copy), the block scales of both in tensor memory
+  static constexpr bool W4A4 = is_w4a4(FMT);
+  static constexpr bool MXS = (FMT == FMT_W4A4MX);   // E8M0 scales per 32 (else E4M3 per 16)
+  // x quantized beforehand: x arrives as codes (e4m3 [M, K] for static FP8,
+  // packed E2M1 for W4A4) through a 2-D u8 map (box 128 bytes x BN rows),
+  // straight into the operand buffer
+  static constexpr bool XQ = (FMT == FMT_FP8SQ) || W4A4;
   static constexpr bool MLP = (FMT == FMT_MLP);
-  static constexpr bool STATIC = (FMT == FMT_FP8S) || XQ || MLP;
+  static constexpr bool STATIC = (FMT == FMT_FP8S) || (FMT == FMT_FP8SQ) || MLP;
+  static constexpr bool SS = STATIC || W4A4;   // A (weight) from shared memory as well
   static constexpr int CHUNK = chunk_bytes(MLP ? FMT_FP8S : FMT);
   static constexpr int X_BYTES = XQ ? 0 : BN * 256;        // two 64-k blocks of BN rows x 128 B
-  static constexpr int Q_BYTES = STATIC ? BN * 128 : 0;    // e4m3 x tile (static FP8)
+  static constexpr int Q_BYTES = SS ? BN * 128 : 0;        // e4m3 / packed E2M1 x tile
+  static constexpr int XSF_BYTES = W4A4 ? 4 * BN * 4 : 0;  // W4A4: x block-scale words [4][BN]
   // Two rings: packed weight chunks (streamed from the start of the kernel;
-  // a slot is free once the prologue has read it, or for static FP8 once the
-  // MMAs have) and x tiles (loaded only after the grid-dependency wait; a
-  // slot is free once the MMAs have read it).
-  static constexpr int X_SLOT = align_up(X_BYTES, 1024) + align_up(Q_BYTES, 1024);
+  // a slot is free once the prologue has read it, or for static FP8 and
+  // W4A4 once the MMAs have) and x tiles (loaded only after the
+  // grid-dependency wait; a slot is free once the MMAs have read it).
+  static constexpr int X_SLOT = align_up(X_BYTES, 1024) + align_up(Q_BYTES + XSF_BYTES, 1024);
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);    // within an x slot
+  static constexpr int XSF_OFF = Q_OFF + Q_BYTES;
   static constexpr int W_SLOT = align_up(CHUNK, 1024);
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
@@ -135,10 +149,16 @@ struct GemmCfg {
   // (a 256-row x tile needs one issuer only: an N = 256 MMA keeps the tensor
   // pipe busy for longer than a thread takes to issue the next)
   static constexpr int ISSUERS = BN >= 256 ? 1 : 2;
-  // k-steps (of 16 bf16 / 32 e4m3) per stage each issuer takes
-  static constexpr int KK = (STATIC ? 4 : 8) / ISSUERS;
-  static constexpr int A_STAGES = STATIC ? 0 : (BN == 64 ? 2 : 3);
-  static constexpr int A_COLS = A_STAGES * (STAGE_K / 2);
+  // k-steps (of 16 bf16 / 32 e4m3 / 64 E2M1) per stage each issuer takes
+  static constexpr int KK = (SS ? 4 : 8) / ISSUERS;
+  // W4A4: the TMEM slots are the stage's block scales instead of operands:
+  // per k-step t, 4 columns for the 128 weight rows (row m at lane m % 32 of
+  // every quadrant, column m / 32) and SFB_COLS for the BN x rows likewise
+  static constexpr int SFB_COLS = BN / 32 < 4 ? 4 : BN / 32;
+  static constexpr int SF_SLOT = 4 * 4 + 4 * SFB_COLS;
+  static constexpr int SFB_OFF = 16;   // within a scale slot
+  static constexpr int A_STAGES = W4A4 ? 3 : STATIC ? 0 : (BN == 64 ? 2 : 3);
+  static constexpr int A_COLS = A_STAGES * (W4A4 ? SF_SLOT : STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
   static constexpr int ACC2_COL = ACC_COL + ISSUERS * BN;   // MLP: layer 2's accumulators
   static constexpr int TMEM_COLS = pow2_at_least(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN);
@@ -149,13 +169,14 @@ struct GemmCfg {
   static constexpr int EPI_OFF = BAR_OFF + BAR_BYTES;
   static constexpr int EPI_BYTES = 2 * 256 * 4;
   static constexpr int SMEM = EPI_OFF + EPI_BYTES + 1024;   // + alignment slack
-  static constexpr uint32_t IDESC = STATIC ? idesc_e4m3(BN) : idesc_bf16(BN);
+  static constexpr uint32_t IDESC = W4A4 ? idesc_fp4(BN, MXS) : STATIC ? idesc_e4m3(BN) : idesc_bf16(BN);
   // warp 0 weight producer, 1 and 10 MMA issuers, 2..9 prologue/epilogue,
   // 11 x producer
   static constexpr int THREADS = 384;
   static_assert(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
   static_assert(!(MLP && BN > 64), "the MLP runs x tiles of at most 64 rows");
   static_assert(!(STATIC && !XQ && BN > 128), "the fused static-FP8 tile holds at most 128 x rows");
+  static_assert(!(W4A4 && BN < 32), "W4A4 x tiles hold 32 rows or more (one scale column per 32 rows)");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");   // (two CTAs per SM need <= 113 KB)
   static_assert(A_STAGES <= 8 && XST <= 8 && WST <= 8, "barrier arrays");
   static_assert(RECV_BYTES % 16 == 0 && RECV_OFF % 16 == 0, "16-byte st.async targets");
@@ -326,7 +347,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   if (threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s) {
       mbar_init(&full_w[s], 1);
-      mbar_init(&wempty[s], C::STATIC ? C::ISSUERS : 8);
+      mbar_init(&wempty[s], C::SS ? C::ISSUERS : 8);
       mbar_init(&full_x[s], 1);
       mbar_init(&xempty[s], C::ISSUERS);
       mbar_init(&aready[s], 8);
@@ -416,9 +437,12 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           if (it >= C::XST && !mbar_wait(&xempty[xs], xph ^ 1, ctl())) { ok = false; break; }
           uint8_t* xd = x_ring + xs * C::X_SLOT;
           if constexpr (C::XQ) {
-            // e4m3 codes straight into the operand buffer of the slot
-            mbar_arrive_expect_tx(&full_x[xs], C::Q_BYTES);
-            tma_load_2d(xd + C::Q_OFF, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
+            // codes straight into the operand buffer of the slot (128 bytes
+            // of each row per stage), and for W4A4 the stage's scale words
+            mbar_arrive_expect_tx(&full_x[xs], C::Q_BYTES + C::XSF_BYTES);
+            tma_load_2d(xd + C::Q_OFF, &tmap_x, ks * 128, m_tile * BN, &full_x[xs]);
+            if constexpr (C::W4A4)
+              bulk_g2s(xd + C::XSF_OFF, p.xsf + ((size_t)m_tile * KS + ks) * 4 * BN, C::XSF_BYTES, &full_x[xs]);
           } else {
             mbar_arrive_expect_tx(&full_x[xs], C::X_BYTES);
             if (p.x3d) {
@@ -452,7 +476,33 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         tc_fence_after();
         for (int j = 0; j < nst; ++j) {
           const uint32_t xb = smem_u32(x_ring + xs * C::X_SLOT);
-          if constexpr (!C::STATIC) {
+          if constexpr (C::W4A4) {
+            // both operands in shared memory (k-step t = 32 bytes into each
+            // 128-byte row), the stage's block scales in TMEM slot `as`
+            if (!mbar_wait(&full_w[ws], wph, ctl()) || !mbar_wait(&full_x[xs], xph, ctl()) ||
+                !mbar_wait(&aready[as], aph, ctl())) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t wb = smem_u32(w_ring + ws * C::W_SLOT) + which * KK * 32;
+            const uint32_t qb = xb + C::Q_OFF + which * KK * 32;
+            const uint32_t sf = tmem + as * C::SF_SLOT;
+#pragma unroll
+            for (int kk = 0; kk < KK; ++kk) {
+              const int t = which * KK + kk;
+              mma_fp4_ss<C::MXS>(d_tmem, sdesc_sw128(wb + kk * 32), sdesc_sw128(qb + kk * 32), C::IDESC, sf + 4 * t,
+                                 sf + C::SFB_OFF + C::SFB_COLS * t, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            issued = true;
+            tc_commit(&wempty[ws]);
+            tc_commit(&aempty[as]);
+            if (++ws == C::WST) {
+              ws = 0;
+              wph ^= 1;
+            }
+            if (++as == C::A_STAGES) {
+              as = 0;
+              aph ^= 1;
+            }
+          } else if constexpr (!C::STATIC) {
             if (!mbar_wait(&full_x[xs], xph, ctl()) || !mbar_wait(&aready[as], aph, ctl())) { ok = false; break; }
             tc_fence_after();
             const uint32_t a_tmem = tmem + as * (STAGE_K / 2) + which * KK * 8;
@@ -549,10 +599,58 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           if (p.col_scale) e_sig = p.sigma * ld_nc_f32(p.col_scale + n_row);
           if (p.bias) e_bias = ld_nc_bf16(p.bias + n_row);
         }
+        if constexpr (FMT == FMT_W4A4NV) {
+          // the activation's global scale is this call's quantizer output:
+          // read only once that grid has completed (and past any cache)
+          pdl_wait();
+          e_sig *= *reinterpret_cast<const volatile float*>(p.gx);
+        }
         epi[et] = e_sig;
         epi[256 + et] = e_bias;
       }
-      if constexpr (!C::STATIC) {
+      if constexpr (C::W4A4) {
+        // the stage's block scales into TMEM slot `as`: every lane quadrant
+        // holds all rows (lane i, column c = row 32c + i); this warp writes
+        // the k-steps t = 2h, 2h + 1 into its own quadrant, from the weight
+        // chunk's and the x slot's scale words ([t][row] each)
+        constexpr int NB = BN / 32;
+        for (int j = 0; j < nst; ++j) {
+          if (!mbar_wait_warp(&full_w[ws], wph, ctl()) || !mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
+          const uint32_t* wsf = reinterpret_cast<const uint32_t*>(w_ring + ws * C::W_SLOT + W4_SF_OFF);
+          const uint32_t* xsf = reinterpret_cast<const uint32_t*>(x_ring + xs * C::X_SLOT + C::XSF_OFF);
+          uint32_t va[8], vb[2 * NB];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = 2 * h + u;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) va[u * 4 + c] = wsf[t * TILE_N + c * 32 + lane];
+#pragma unroll
+            for (int c = 0; c < NB; ++c) vb[u * NB + c] = xsf[t * BN + c * 32 + lane];
+          }
+          if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ts = tmem + lane_base + as * C::SF_SLOT;
+          tmem_st_cols<8>(ts + 8 * h, va);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) tmem_st_cols<NB>(ts + C::SFB_OFF + C::SFB_COLS * (2 * h + u), vb + u * NB);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&aready[as]);
+          if (++ws == C::WST) {
+            ws = 0;
+            wph ^= 1;
+          }
+          if (++xs == C::XST) {
+            xs = 0;
+            xph ^= 1;
+          }
+          if (++as == C::A_STAGES) {
+            as = 0;
+            aph ^= 1;
+          }
+        }
+      } else if constexpr (!C::STATIC) {
         // the weight operand needs no x: the first A_STAGES stages are
         // unpacked before the grid-dependency wait has even returned
         for (int j = 0; j < nst; ++j) {

@@ -35,6 +35,13 @@
 // in the epilogue).  Static-FP8 chunks are the tensor core's K-major,
 // 128-byte-swizzled shared-memory image of the 128 x 128 e4m3 tile:
 //   byte (r, k) at r*128 + (((k >> 4) ^ (r & 7)) << 4) + (k & 15).
+// FP4 x FP4 (W4A4) chunks cover 256 k per stage: the 128 x 128-byte image of
+// the packed E2M1 codes in the same swizzled layout (byte b of a row holds
+// k = 2b in its low nibble and k = 2b + 1 in its high nibble), then the block
+// scales as tensor-memory words, one per (k-step t of 64, row r) at
+// 16384 + (t * 128 + r) * 4:
+//   MXFP4 (E8M0 per 32)  byte 0 = block 2t, byte 1 = block 2t + 1, bytes 2-3 zero
+//   NVFP4 (E4M3 per 16)  byte j = block 4t + j
 #pragma once
 
 #include <stdint.h>
@@ -43,6 +50,9 @@ namespace dq {
 
 enum Fmt { FMT_INT4 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_FP8S = 4,
            FMT_INT4A = 5,   // asymmetric INT4, per-group zero point
+           // FP4 x FP4 with dynamic activation quantization (native
+           // block-scaled MMA): MXFP4 and NVFP4 weights
+           FMT_W4A4MX = 6, FMT_W4A4NV = 7,
            // static FP8 GEMM fed with activations quantized beforehand (same
            // weight chunks as FMT_FP8S; a kernel variant, not a storage format)
            FMT_FP8SQ = 8,
@@ -53,9 +63,14 @@ enum Fmt { FMT_INT4 = 0, FMT_NVFP4 = 1, FMT_MXFP4 = 2, FMT_FP8 = 3, FMT_FP8S = 4
 constexpr int TILE_N = 128;      // output channels per tile (MMA M)
 constexpr int STAGE_K = 128;     // k per pipeline stage (= one INT4 group)
 constexpr int PACKED4_BYTES = TILE_N * STAGE_K / 2;   // 8192
+constexpr int W4_STAGE_K = 256;  // k per pipeline stage of the FP4 x FP4 GEMM (128 bytes of codes a row)
+constexpr int W4_SF_OFF = TILE_N * W4_STAGE_K / 2;    // 16384: the scale words of a W4A4 chunk
+
+__host__ __device__ constexpr bool is_w4a4(int fmt) { return fmt == FMT_W4A4MX || fmt == FMT_W4A4NV; }
 
 __host__ __device__ constexpr int chunk_bytes(int fmt) {
-  return fmt == FMT_INT4 ? PACKED4_BYTES + TILE_N * 2
+  return is_w4a4(fmt) ? W4_SF_OFF + 4 * TILE_N * 4
+       : fmt == FMT_INT4 ? PACKED4_BYTES + TILE_N * 2
        : fmt == FMT_INT4A ? PACKED4_BYTES + TILE_N * 3
        : fmt == FMT_NVFP4 ? PACKED4_BYTES + TILE_N * 8
        : fmt == FMT_MXFP4 ? PACKED4_BYTES + TILE_N * 4
