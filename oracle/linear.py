@@ -11,8 +11,7 @@ Format names used here and by the tests:
   "fp8_static" E4M3 weights and activations (static FP8 page)
 
 The FP4 x FP4 section at the end (dynamic activation quantization and the
-W4A4 reference) is the native-MMA variant the MXFP4 page names; the library
-has no kernel for it yet.
+W4A4 reference) is the native-MMA variant the MXFP4 page names.
 """
 
 import numpy as np
@@ -222,7 +221,7 @@ def sqnr(a, b):
 # ---------------------------------------------------------------------------
 # FP4 x FP4 ("TorchAO MXFP4 Dynamic Activation + MX Weight (Linear)", intro:
 # the config is MX dynamic activation + MX weight, and native MXFP4 x MXFP4
-# needs B200).  Not served by the library yet; the reference of that path.
+# needs B200): the reference of that path.
 # ---------------------------------------------------------------------------
 
 

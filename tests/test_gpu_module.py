@@ -87,7 +87,8 @@ def test_layer_rejects_bad_tensors_before_launch():
     lin.close()
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4", "fp8", "int4_asym", "fp8_static"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4", "fp8", "int4_asym", "fp8_static", "w4a4_mxfp4",
+                                 "w4a4_nvfp4"])
 def test_quantized_module_matches_oracle(fmt):
     """The pages' flow end to end against the fp64 oracle: a bf16
     nn.Linear(3072, 512) quantized in place by quantize_, called on x with
@@ -99,7 +100,7 @@ def test_quantized_module_matches_oracle(fmt):
 
     from oracle import linear as L
 
-    from gpu_util import bf16_values, check_close, static_effective_x
+    from gpu_util import base_fmt, bf16_values, check_close, static_effective_x
 
     torch.manual_seed(7)
     model = torch.nn.Sequential(torch.nn.Linear(3072, 512)).to(device="cuda", dtype=torch.bfloat16)
@@ -114,9 +115,17 @@ def test_quantized_module_matches_oracle(fmt):
         y = model(x)
     torch.cuda.synchronize()
     assert model[0].layer.last_error() == 0
-    base = "fp8" if fmt == "fp8_static" else fmt
+    base = base_fmt(fmt)
     st = L.quantize_pack(base, W)
     wdq = L.dequant_exact(base, st["packed"], st["scales"], st["global_scale"])
     xv = bf16_values(x.view(-1, 3072))
-    x_eff = static_effective_x(xv, scales["0"]) if fmt == "fp8_static" else xv
-    check_close(bf16_values(y.view(-1, 512)), L.linear_ref(x_eff, wdq, b), x_eff, wdq)
+    if fmt.startswith("w4a4"):
+        # W4A4: the activations are quantized per call with the weight's recipe
+        from gpu_util import w4a4_effective_x
+
+        x_eff = w4a4_effective_x(fmt, xv)
+        ref = L.w4a4_linear_ref(base, xv, st["packed"], st["scales"], st["global_scale"], b)
+    else:
+        x_eff = static_effective_x(xv, scales["0"]) if fmt == "fp8_static" else xv
+        ref = L.linear_ref(x_eff, wdq, b)
+    check_close(bf16_values(y.view(-1, 512)), ref, x_eff, wdq)

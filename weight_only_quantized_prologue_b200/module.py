@@ -19,7 +19,7 @@ import torch
 
 from . import QuantizedLinear
 
-FORMATS = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static", "int4_asym")
+FORMATS = ("int4", "nvfp4", "mxfp4", "fp8", "fp8_static", "int4_asym", "w4a4_mxfp4", "w4a4_nvfp4")
 
 # live layers by handle value, so the op can reach the Python object (the
 # static-FP8 path needs its activation scale and K)
