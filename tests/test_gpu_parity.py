@@ -96,6 +96,38 @@ def test_quantize_act_fp8_bit_exact():
     assert np.array_equal(q.cpu().numpy(), ref)
 
 
+def _all_finite_bf16():
+    """Every finite bf16 bit pattern (65,024 of the 65,536; NaN and inf
+    patterns become zeros), as a [256, 256] tensor."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = (bits & 0x7F80) != 0x7F80
+    bits = np.where(finite, bits, 0).astype(np.uint16)
+    return torch.from_numpy(bits.view(np.int16).reshape(256, 256).copy()).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("s_x", [0.0123, 3.0, 1.0 / 3.0, 7.77e-6, 2.5e4, 1.0e-30, 0.1])
+def test_quantize_act_fp8_every_bf16_value(s_x):
+    # the quantizer forms f32(x / s_x) without dividing (a multiply by the
+    # reciprocal and one correction step); its codes must equal those of the
+    # exact quotient for every bf16 input, both kernels (vector, and
+    # element-wise through an unaligned buffer)
+    s_x = float(np.float32(s_x))
+    x = _all_finite_bf16()
+    ref = L.quantize_act_fp8(bf16_values(x), s_x)
+    q = torch.empty((256, 256), dtype=torch.uint8, device="cuda")
+    dq.dqgemm_quantize_act_fp8(x.cuda(), 256, 256, s_x, q)
+    xe = torch.zeros(65537, dtype=torch.bfloat16, device="cuda")
+    xe[1:] = x.view(-1).cuda()
+    qe = torch.zeros(65537, dtype=torch.uint8, device="cuda")
+    assert dq._native.lib().dqgemm_quantize_act_fp8(xe.data_ptr() + 2, 256, 256, s_x, qe.data_ptr() + 1, None) == 0
+    torch.cuda.synchronize()
+    got = q.cpu().numpy()
+    bad = np.argwhere(got != ref)
+    assert bad.size == 0, (f"{len(bad)} codes differ, e.g. x bits {x.view(torch.int16)[tuple(bad[0])].item() & 0xFFFF:#06x}: "
+                           f"{got[tuple(bad[0])]:#04x} vs {ref[tuple(bad[0])]:#04x}")
+    assert np.array_equal(qe.cpu().numpy()[1:].reshape(256, 256), ref)
+
+
 @pytest.mark.parametrize("M,K,offset", [(5, 19, 0), (129, 4096, 0), (3, 272, 1), (64, 1000, 3)])
 def test_quantize_act_fp8_vector_tail_and_unaligned(M, K, offset):
     # 16 elements per thread where x and q are 16-byte aligned, element-wise

@@ -561,6 +561,14 @@ bool x_map(dqgemm_s* h, const void* x, int M, int bn, bool xq, CUtensorMap* tm, 
 
 dqgemm_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA; }
 
+// f32(1 / s), correctly rounded (an IEEE fp32 division on the host): the
+// reciprocal the kernels' static-FP8 quantizers multiply by
+float recip_rn(float s) {
+  volatile float one = 1.f;
+  volatile float r = one / s;
+  return r;
+}
+
 // a small kernel in the programmatic-dependent-launch chain of the GEMMs
 // (its first instruction waits for the previous grid)
 template <typename... KArgs, typename... Args>
@@ -805,6 +813,8 @@ static dqgemm_status run_w4a4(dqgemm_handle h, const void* x, int M, void* y, vo
   p.sigma = h->sigma;
   p.s_x = 1.f;
   p.s_out = 1.f;
+  p.r_x = 1.f;
+  p.r_out = 1.f;
   p.M = M;
   p.N = h->N;
   p.k_stages = h->k_stages;
@@ -841,9 +851,11 @@ static dqgemm_status run_gemm(dqgemm_handle h, const void* x, bool xq, int M, vo
   p.y = yq ? nullptr : static_cast<__nv_bfloat16*>(y);
   p.yq = yq ? static_cast<uint8_t*>(y) : nullptr;
   p.s_out = yq ? s_out : 1.f;
+  p.r_out = recip_rn(p.s_out);
   p.status = h->status;
   p.sigma = h->sigma;
   p.s_x = h->s_x;
+  p.r_x = recip_rn(p.s_x);
   p.mx_bias = h->mx_bias;
   p.M = M;
   p.N = h->N;
@@ -909,6 +921,8 @@ dqgemm_status dqgemm_run_static_mlp(dqgemm_handle l1, dqgemm_handle l2, const vo
   p.sigma = l1->s_x;
   p.s_x = l1->s_x;
   p.s_out = l2->s_x;
+  p.r_x = recip_rn(p.s_x);
+  p.r_out = recip_rn(p.s_out);
   p.M = M;
   p.N = l1->N;
   p.k_stages = l1->k_stages;

@@ -51,18 +51,33 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* wchunks, co
 // ---------------------------------------------------------------------------
 // static FP8 activation quantization: q = e4m3(f32(x / s_x)), saturating
 // ---------------------------------------------------------------------------
-__global__ void act_quant_kernel(const __nv_bfloat16* x, long long count, float s_x, uint8_t* q) {
+template <bool FAST>
+__device__ __forceinline__ uint32_t act_code_t(float v, float s, float r) {
+  return e4m3_code(FAST ? e4m3_quotient(v, s, r) : __fdiv_rn(v, s));
+}
+
+template <bool FAST>
+__device__ __forceinline__ void act_quant_loop(const __nv_bfloat16* x, long long count, float s_x, float r_x,
+                                               uint8_t* q) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
-       i += (long long)gridDim.x * blockDim.x) {
-    q[i] = act_code(__bfloat162float(x[i]), s_x);
-  }
+       i += (long long)gridDim.x * blockDim.x)
+    q[i] = (uint8_t)act_code_t<FAST>(__bfloat162float(x[i]), s_x, r_x);
+}
+
+__global__ void act_quant_kernel(const __nv_bfloat16* x, long long count, float s_x, uint8_t* q) {
+  const float r_x = __frcp_rn(s_x);
+  if (e4m3_quotient_ok(r_x))
+    act_quant_loop<true>(x, count, s_x, r_x, q);
+  else
+    act_quant_loop<false>(x, count, s_x, r_x, q);
 }
 
 // The same, 16 elements per thread: two 16-byte loads of bf16, one 16-byte
 // store of codes (x and q 16-byte aligned; `groups` = count / 16, the tail
-// goes to act_quant_kernel).  Each code is act_code of the same value,
-// so the result is bit-identical with the element-wise kernel.
-__global__ void act_quant16_kernel(const uint4* x, long long groups, float s_x, uint4* q) {
+// goes to act_quant_kernel).  Each code is the same function of the same
+// value, so the result is bit-identical with the element-wise kernel.
+template <bool FAST>
+__device__ __forceinline__ void act_quant16_loop(const uint4* x, long long groups, float s_x, float r_x, uint4* q) {
   for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < groups;
        g += (long long)gridDim.x * blockDim.x) {
     const uint4 a = x[2 * g], b = x[2 * g + 1];
@@ -74,14 +89,22 @@ __global__ void act_quant16_kernel(const uint4* x, long long groups, float s_x, 
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const uint32_t v = in[2 * w + k];
-        const uint32_t lo = act_code(__uint_as_float(v << 16), s_x);
-        const uint32_t hi = act_code(__uint_as_float(v & 0xFFFF0000u), s_x);
+        const uint32_t lo = act_code_t<FAST>(__uint_as_float(v << 16), s_x, r_x);
+        const uint32_t hi = act_code_t<FAST>(__uint_as_float(v & 0xFFFF0000u), s_x, r_x);
         word |= (lo | (hi << 8)) << (16 * k);
       }
       out[w] = word;
     }
     q[g] = make_uint4(out[0], out[1], out[2], out[3]);
   }
+}
+
+__global__ void act_quant16_kernel(const uint4* x, long long groups, float s_x, uint4* q) {
+  const float r_x = __frcp_rn(s_x);
+  if (e4m3_quotient_ok(r_x))
+    act_quant16_loop<true>(x, groups, s_x, r_x, q);
+  else
+    act_quant16_loop<false>(x, groups, s_x, r_x, q);
 }
 
 // ---------------------------------------------------------------------------

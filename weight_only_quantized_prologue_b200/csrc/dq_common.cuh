@@ -246,11 +246,35 @@ __device__ __forceinline__ uint8_t e4m3_code(float v) {
   return c;
 }
 
+// f32(v / s), correctly rounded, for the e4m3 conversion that follows,
+// without a division: Markstein's correction step (P. Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", 1990).
+// With r = f32(1 / s) correctly rounded, q0 = f32(v * r) lies within one
+// unit in the last place of v / s, the residual v - q0 * s is then exact in
+// one fused multiply-add, and f32(q0 + residual * r) is the correctly
+// rounded quotient, provided nothing overflows or underflows.  Outside
+// [2^-12, 2^9) the e4m3 code is +-0 or +-448 whatever the quotient's last
+// bits, so q0 is used as it is there (which also keeps the residual in
+// range).  r must be a normal fp32 value (s within [2^-126, 2^126]).
+__device__ __forceinline__ float e4m3_quotient(float v, float s, float r) {
+  const float q0 = __fmul_rn(v, r);
+  const float a = fabsf(q0);
+  if (!(a >= 0x1p-12f && a < 0x1p9f)) return q0;
+  return __fmaf_rn(__fmaf_rn(-q0, s, v), r, q0);
+}
+
+// whether e4m3_quotient may be used for the scale s (its reciprocal normal)
+__device__ __forceinline__ bool e4m3_quotient_ok(float r) {
+  const uint32_t e = __float_as_uint(r) & 0x7F800000u;
+  return e != 0u && e != 0x7F800000u;
+}
+
 // static-FP8 activation code of a value v (the Q node): e4m3(f32(v / s)),
-// IEEE division; a zero v gives its signed zero code without dividing
-// (the division is slow for a zero dividend, and exact either way)
-__device__ __forceinline__ uint8_t act_code(float v, float s) {
-  return v == 0.f ? (signbit(v) ? 0x80 : 0x00) : e4m3_code(__fdiv_rn(v, s));
+// the IEEE quotient (r = f32(1 / s); the division itself where r is not a
+// normal number)
+__device__ __forceinline__ uint8_t act_code_r(float v, float s, float r) {
+  if (e4m3_quotient_ok(r)) return e4m3_code(e4m3_quotient(v, s, r));
+  return e4m3_code(__fdiv_rn(v, s));
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -298,6 +322,18 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// e4m3 x e4m3 with A (128 x 32 e4m3, four codes a 32-bit column, the lower
+// k in the lower byte) in tensor memory and B in shared memory
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

@@ -47,6 +47,7 @@ struct GemmParams {
   int* status;                   // device status word
   float sigma;                   // epilogue factor common to all channels
   float s_x;                     // static FP8 activation scale
+  float r_x, r_out;              // f32(1 / s_x) and f32(1 / s_out), correctly rounded (host division)
   int mx_bias;                   // MXFP4: 126 - J
   int M, N, k_stages, m_tiles;
   int tiles;                     // n_tiles * m_tiles
@@ -77,7 +78,7 @@ struct GemmParams {
 // q = e4m3(f32(bf16(v)) / s_out): the code dqgemm_quantize_act_fp8 gives
 // for the bf16 output y = bf16(v)
 __device__ __forceinline__ uint8_t out_code(const GemmParams& p, float v) {
-  return act_code(__bfloat162float(__float2bfloat16_rn(v)), p.s_out);
+  return act_code_r(__bfloat162float(__float2bfloat16_rn(v)), p.s_out, p.r_out);
 }
 
 __host__ __device__ constexpr int align_up(int v, int a) { return (v + a - 1) / a * a; }
@@ -98,22 +99,33 @@ struct GemmCfg {
   static constexpr bool XQ = (FMT == FMT_FP8SQ) || W4A4;
   static constexpr bool MLP = (FMT == FMT_MLP);
   static constexpr bool STATIC = (FMT == FMT_FP8S) || (FMT == FMT_FP8SQ) || MLP;
-  static constexpr bool SS = STATIC || W4A4;   // A (weight) from shared memory as well
+  // fused static FP8: the e4m3 weight stage is copied from shared memory into
+  // a ring of TMEM slots (32 columns each) and the MMA reads A there, so the
+  // weight slots are free again at once and many stages stream in before the
+  // grid-dependency wait (A from shared memory would hold every stage's slot
+  // until its MMAs complete)
+  static constexpr bool TSA = (FMT == FMT_FP8S);
+  static constexpr bool SS = (STATIC && !TSA) || W4A4;   // A (weight) from shared memory as well
   static constexpr int CHUNK = chunk_bytes(MLP ? FMT_FP8S : FMT);
   static constexpr int X_BYTES = XQ ? 0 : BN * 256;        // two 64-k blocks of BN rows x 128 B
-  static constexpr int Q_BYTES = SS ? BN * 128 : 0;        // e4m3 / packed E2M1 x tile
+  static constexpr int Q_BYTES = (STATIC || W4A4) ? BN * 128 : 0;   // e4m3 / packed E2M1 x tile
   static constexpr int XSF_BYTES = W4A4 ? 4 * BN * 4 : 0;  // W4A4: x block-scale words [4][BN]
   // Two rings: packed weight chunks (streamed from the start of the kernel;
   // a slot is free once the prologue has read it, or for static FP8 and
   // W4A4 once the MMAs have) and x tiles (loaded only after the
   // grid-dependency wait; a slot is free once the MMAs have read it).
-  static constexpr int X_SLOT = align_up(X_BYTES, 1024) + align_up(Q_BYTES + XSF_BYTES, 1024);
+  // (fused static FP8 with A in TMEM keeps the bf16 x tiles and their e4m3
+  // operands in separate rings: a bf16 slot is free as soon as its tile is
+  // quantized, an operand slot once the MMAs have read it)
+  static constexpr int X_SLOT = TSA ? align_up(X_BYTES, 1024) : align_up(X_BYTES, 1024) + align_up(Q_BYTES + XSF_BYTES, 1024);
+  static constexpr int Q_SLOT = align_up(Q_BYTES, 1024);
   static constexpr int Q_OFF = align_up(X_BYTES, 1024);    // within an x slot
   static constexpr int XSF_OFF = Q_OFF + Q_BYTES;
   static constexpr int W_SLOT = align_up(CHUNK, 1024);
   // skinny tiles keep a CTA under half an SM's shared memory so that the next
   // call's CTA can be resident alongside (programmatic dependent launch)
-  static constexpr int SMEM_BUDGET = BN <= 64 ? 108 * 1024 : (BN <= 128 ? 200 * 1024 : 216 * 1024);
+  static constexpr int SMEM_BUDGET = TSA ? (BN <= 32 ? 108 * 1024 : 216 * 1024)
+                                         : BN <= 64 ? 108 * 1024 : (BN <= 128 ? 200 * 1024 : 216 * 1024);
   // split-K receive area: the S partials (its own included) of the columns
   // this CTA owns, [rank][row][BN / S] fp32 = one 128 x BN fp32 tile, then
   // one validity word per (rank, 32 rows) (256-row x tiles run whole tiles
@@ -128,15 +140,26 @@ struct GemmCfg {
   // The x ring is as deep as the budget allows while keeping three weight
   // slots: a skinny split CTA (six 128-k stages at 32 x 3072 x 4096) then
   // issues every x load of its k-range right after the grid-dependency wait.
-  static constexpr int XST = (AVAIL - 6 * X_SLOT >= 3 * W_SLOT)   ? 6
+  // (TSA: the weights drain into TMEM at once, so two or three weight slots
+  // do; the bf16 landing ring gets as many slots as leave the operand ring
+  // 4 (2 from 64 rows on), up to 8, so that most x loads of a CTA's k-range
+  // are issued together after the grid-dependency wait; the operand ring
+  // takes the rest, up to 8)
+  static constexpr int TSA_WST = BN <= 16 ? 3 : 2;
+  static constexpr int TSA_XST = (AVAIL - TSA_WST * W_SLOT - (BN <= 32 ? 4 : 2) * Q_SLOT) / (X_SLOT > 0 ? X_SLOT : 1);
+  static constexpr int XST = TSA ? (TSA_XST > 8 ? 8 : TSA_XST < 2 ? 2 : TSA_XST)
+                             : (AVAIL - 6 * X_SLOT >= 3 * W_SLOT) ? 6
                              : (AVAIL - 4 * X_SLOT >= 3 * W_SLOT) ? 4
                              : (AVAIL - 3 * X_SLOT >= 3 * W_SLOT) ? 3
                                                                   : 2;
-  static constexpr int WST_RAW = (AVAIL - XST * X_SLOT) / W_SLOT;
+  static constexpr int WST_RAW = TSA ? TSA_WST : (AVAIL - XST * X_SLOT) / W_SLOT;
   static constexpr int WST = WST_RAW < 2 ? 2 : (WST_RAW > 8 ? 8 : WST_RAW);
+  static constexpr int QST_RAW = TSA ? (AVAIL - XST * X_SLOT - WST * W_SLOT) / Q_SLOT : 0;
+  static constexpr int QST = QST_RAW > 8 ? 8 : QST_RAW;
   static constexpr int STAGES = WST;   // weight stages in flight (reported by the plan)
   static constexpr int X_RING_OFF = 0;
-  static constexpr int W_RING_OFF = XST * X_SLOT;
+  static constexpr int Q_RING_OFF = XST * X_SLOT;
+  static constexpr int W_RING_OFF = Q_RING_OFF + QST * Q_SLOT;
   static constexpr int RECV_OFF = W_RING_OFF + WST * W_SLOT;
   static constexpr int RFLAG_OFF = RECV_OFF + RECV_BYTES;
   static constexpr int W2_OFF = align_up(RFLAG_OFF + RFLAG_BYTES, 1024);
@@ -150,20 +173,22 @@ struct GemmCfg {
   // pipe busy for longer than a thread takes to issue the next)
   static constexpr int ISSUERS = BN >= 256 ? 1 : 2;
   // k-steps (of 16 bf16 / 32 e4m3 / 64 E2M1) per stage each issuer takes
-  static constexpr int KK = (SS ? 4 : 8) / ISSUERS;
+  static constexpr int KK = (SS || TSA ? 4 : 8) / ISSUERS;
   // W4A4: the TMEM slots are the stage's block scales instead of operands:
   // per k-step t, 4 columns for the 128 weight rows (row m at lane m % 32 of
   // every quadrant, column m / 32) and SFB_COLS for the BN x rows likewise
   static constexpr int SFB_COLS = BN / 32 < 4 ? 4 : BN / 32;
   static constexpr int SF_SLOT = 4 * 4 + 4 * SFB_COLS;
   static constexpr int SFB_OFF = 16;   // within a scale slot
-  static constexpr int A_STAGES = W4A4 ? 3 : STATIC ? 0 : (BN == 64 ? 2 : 3);
-  static constexpr int A_COLS = A_STAGES * (W4A4 ? SF_SLOT : STAGE_K / 2);
+  // (TSA: every TMEM column the accumulators leave, at most 8 slots)
+  static constexpr int TSA_STAGES = ((BN <= 64 ? 256 : 512) - 2 * BN) / 32 > 8 ? 8 : ((BN <= 64 ? 256 : 512) - 2 * BN) / 32;
+  static constexpr int A_STAGES = W4A4 ? 3 : TSA ? TSA_STAGES : STATIC ? 0 : (BN == 64 ? 2 : 3);
+  static constexpr int A_COLS = A_STAGES * (W4A4 ? SF_SLOT : TSA ? STAGE_K / 4 : STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
   static constexpr int ACC2_COL = ACC_COL + ISSUERS * BN;   // MLP: layer 2's accumulators
   static constexpr int TMEM_COLS = pow2_at_least(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN);
   static constexpr int BAR_OFF = B2_OFF + B2_BYTES;
-  static constexpr int BAR_BYTES = 8 * 64;
+  static constexpr int BAR_BYTES = 8 * 80;
   // each epilogue thread's row factor and bias, parked in shared memory over
   // the main loop instead of holding registers: [2][256] fp32
   static constexpr int EPI_OFF = BAR_OFF + BAR_BYTES;
@@ -179,6 +204,7 @@ struct GemmCfg {
   static_assert(!(W4A4 && BN < 32), "W4A4 x tiles hold 32 rows or more (one scale column per 32 rows)");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");   // (two CTAs per SM need <= 113 KB)
   static_assert(A_STAGES <= 8 && XST <= 8 && WST <= 8, "barrier arrays");
+  static_assert(!TSA || QST >= 2, "operand ring");
   static_assert(RECV_BYTES % 16 == 0 && RECV_OFF % 16 == 0, "16-byte st.async targets");
 };
 
@@ -280,10 +306,12 @@ __device__ __forceinline__ void prologue_stage(const uint8_t* chunk, int r, int 
 }
 
 // Static FP8: quantize the bf16 x tile (two SW128 boxes) into the e4m3 SW128
-// B operand: q = e4m3(f32(x / s_x)), IEEE division, RNE, saturating.
-template <int BN>
-__device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, float s_x, int tid) {
-  for (int c = tid; c < BN * 8; c += 256) {
+// B operand: q = e4m3(f32(x / s_x)), the IEEE quotient, RNE, saturating.
+// (FAST: the quotient by e4m3_quotient; a separate loop, so the division is
+// not evaluated alongside)
+template <int BN, int NT, bool FAST>
+__device__ __forceinline__ void quantize_x_tile_loop(const uint8_t* xs, uint8_t* qs, float s_x, float r_x, int tid) {
+  for (int c = tid; c < BN * 8; c += NT) {
     const int row = c >> 3, cc = c & 7;
     const uint8_t* box = xs + (cc >> 2) * BN * 128 + row * 128;
     const uint4 a = lds128(box + (((2 * (cc & 3)) ^ (row & 7)) << 4));
@@ -297,15 +325,22 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
       for (int k = 0; k < 2; ++k) {
         const uint32_t w = in[2 * i + k];
         const float f0 = __uint_as_float(w << 16), f1 = __uint_as_float(w & 0xFFFF0000u);
-        // (+-0 / s_x is +-0: no division, which is slow for a zero dividend;
-        // at one activation row 15 of a 16-row tile are the TMA's zero fill)
-        const float2 qv = make_float2(f0 == 0.f ? f0 : __fdiv_rn(f0, s_x), f1 == 0.f ? f1 : __fdiv_rn(f1, s_x));
+        const float2 qv = FAST ? make_float2(e4m3_quotient(f0, s_x, r_x), e4m3_quotient(f1, s_x, r_x))
+                               : make_float2(__fdiv_rn(f0, s_x), __fdiv_rn(f1, s_x));
         lohi[k] = (uint32_t)__nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
       }
       out[i] = lohi[0] | (lohi[1] << 16);
     }
     sts128(qs + row * 128 + ((cc ^ (row & 7)) << 4), make_uint4(out[0], out[1], out[2], out[3]));
   }
+}
+
+template <int BN, int NT = 256>
+__device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, float s_x, float r_x, int tid) {
+  if (e4m3_quotient_ok(r_x))
+    quantize_x_tile_loop<BN, NT, true>(xs, qs, s_x, r_x, tid);
+  else
+    quantize_x_tile_loop<BN, NT, false>(xs, qs, s_x, r_x, tid);
 }
 
 // QOUT: the output leaves as the next static-FP8 layer's e4m3 codes (a
@@ -332,7 +367,9 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint64_t* full_w2 = recv_bar + 1;       // MLP: layer 2's weight chunk landed
   uint64_t* b2ready = full_w2 + 1;        // MLP: layer 2's B operand (hidden codes) written
   uint64_t* acc2_full = b2ready + 1;      // MLP: layer 2's accumulators complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc2_full + 1);
+  uint64_t* xready = acc2_full + 1;       // [8] fused static with A in TMEM: operand slot written
+  uint64_t* qempty = xready + 8;          // [8]   ... and read by the MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);             // [S][128][BN/S]
   uint32_t* rflag = reinterpret_cast<uint32_t*>(smem + C::RFLAG_OFF);     // [S][4]: sender rank, row quadrant
@@ -347,10 +384,12 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   if (threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s) {
       mbar_init(&full_w[s], 1);
-      mbar_init(&wempty[s], C::SS ? C::ISSUERS : 8);
+      mbar_init(&wempty[s], C::SS ? C::ISSUERS : C::TSA ? 4 : 8);
       mbar_init(&full_x[s], 1);
-      mbar_init(&xempty[s], C::ISSUERS);
-      mbar_init(&aready[s], 8);
+      mbar_init(&xempty[s], C::TSA ? 4 : C::ISSUERS);   // (TSA: the quantizing warps free the bf16 slot)
+      mbar_init(&aready[s], C::TSA ? 4 : 8);
+      mbar_init(&xready[s], 4);
+      mbar_init(&qempty[s], C::ISSUERS);
       mbar_init(&aempty[s], C::ISSUERS);
     }
     mbar_init(acc_full, C::ISSUERS);
@@ -519,6 +558,23 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
               as = 0;
               aph ^= 1;
             }
+          } else if constexpr (C::TSA) {
+            // A: the e4m3 weight stage in TMEM slot `as` (8 columns per
+            // k-step of 32); B: the e4m3 operand in slot xs of the operand
+            // ring (xs / xph count that ring here)
+            if (!mbar_wait(&aready[as], aph, ctl()) || !mbar_wait(&xready[xs], xph, ctl())) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_tmem = tmem + as * (STAGE_K / 4) + which * KK * 8;
+            const uint32_t qb = smem_u32(smem + C::Q_RING_OFF + xs * C::Q_SLOT) + which * KK * 32;
+#pragma unroll
+            for (int kk = 0; kk < KK; ++kk)
+              mma_f8_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(qb + kk * 32), C::IDESC, (j > 0 || kk > 0) ? 1u : 0u);
+            issued = true;
+            tc_commit(&aempty[as]);
+            if (++as == C::A_STAGES) {
+              as = 0;
+              aph ^= 1;
+            }
           } else {
             if (!mbar_wait(&full_w[ws], wph, ctl()) || !mbar_wait(&aready[xs], xph, ctl())) { ok = false; break; }
             tc_fence_after();
@@ -535,10 +591,18 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
               wph ^= 1;
             }
           }
-          tc_commit(&xempty[xs]);
-          if (++xs == C::XST) {
-            xs = 0;
-            xph ^= 1;
+          if constexpr (C::TSA) {
+            tc_commit(&qempty[xs]);
+            if (++xs == C::QST) {
+              xs = 0;
+              xph ^= 1;
+            }
+          } else {
+            tc_commit(&xempty[xs]);
+            if (++xs == C::XST) {
+              xs = 0;
+              xph ^= 1;
+            }
           }
         }
         if (!ok) break;
@@ -585,8 +649,8 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     float* epi = reinterpret_cast<float*>(smem + C::EPI_OFF);   // [2][256]: this thread's slots only
     const int et = threadIdx.x - 64;
     int tile = 0;
-    int ws = 0, xs = 0, as = 0;
-    uint32_t wph = 0, xph = 0, aph = 0;
+    int ws = 0, xs = 0, as = 0, qs = 0;     // ring positions, kept across the tiles of a persistent CTA
+    uint32_t wph = 0, xph = 0, aph = 0, qph = 0;
     bool ok = true, have_acc = false;
     for (int t = 0; ok && t < wk.ntiles; ++t) {
       tile = wk.first_tile + t * wk.tile_step;
@@ -650,6 +714,76 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
             aph ^= 1;
           }
         }
+      } else if constexpr (C::TSA) {
+        if (h == 0) {
+          // warps 2..5, one per lane quadrant: weight row r's 128 e4m3 codes
+          // from the swizzled image into TMEM slot `as` (the weights need no
+          // x: these run ahead of the grid-dependency wait, A_STAGES deep)
+          for (int j = 0; j < nst; ++j) {
+            if (!mbar_wait_warp(&full_w[ws], wph, ctl())) { ok = false; break; }
+            // (in two halves of 64 codes, as the unpack does, to keep the
+            // live registers low; the slot is free once the second is read)
+            const uint8_t* row = w_ring + ws * C::W_SLOT + r * 128;
+            const uint32_t ta = tmem + lane_base + as * (STAGE_K / 4);
+            uint32_t o[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 v = lds128(row + ((c ^ (r & 7)) << 4));
+              o[4 * c] = v.x;
+              o[4 * c + 1] = v.y;
+              o[4 * c + 2] = v.z;
+              o[4 * c + 3] = v.w;
+            }
+            if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) { ok = false; break; }
+            tc_fence_after();
+            tmem_st16(ta, o);
+#pragma unroll
+            for (int c = 4; c < 8; ++c) {
+              const uint4 v = lds128(row + ((c ^ (r & 7)) << 4));
+              o[4 * c - 16] = v.x;
+              o[4 * c - 15] = v.y;
+              o[4 * c - 14] = v.z;
+              o[4 * c - 13] = v.w;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wempty[ws]);
+            tmem_st16(ta + 16, o);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&aready[as]);
+            if (++ws == C::WST) {
+              ws = 0;
+              wph ^= 1;
+            }
+            if (++as == C::A_STAGES) {
+              as = 0;
+              aph ^= 1;
+            }
+          }
+        } else {
+          // warps 6..9: quantize each bf16 x tile into a slot of the operand
+          // ring (qs), then free the bf16 slot for the next load
+          for (int j = 0; j < nst; ++j) {
+            if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
+            if (!mbar_wait_warp(&qempty[qs], qph ^ 1, ctl())) { ok = false; break; }
+            quantize_x_tile<BN, 128>(x_ring + xs * C::X_SLOT, smem + C::Q_RING_OFF + qs * C::Q_SLOT, p.s_x, p.r_x, et - 128);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&xready[qs]);
+              mbar_arrive(&xempty[xs]);
+            }
+            if (++xs == C::XST) {
+              xs = 0;
+              xph ^= 1;
+            }
+            if (++qs == C::QST) {
+              qs = 0;
+              qph ^= 1;
+            }
+          }
+        }
       } else if constexpr (!C::STATIC) {
         // the weight operand needs no x: the first A_STAGES stages are
         // unpacked before the grid-dependency wait has even returned
@@ -690,7 +824,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
           if constexpr (!C::XQ) {
             uint8_t* xd = x_ring + xs * C::X_SLOT;
-            quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, et);
+            quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, p.r_x, et);
             fence_proxy_async_smem();
           }
           __syncwarp();
