@@ -71,6 +71,30 @@ def test_activation_quantizer_bit_exact(fmt, M, K):
     assert np.array_equal(c, pack_nibbles(rc)), f"{(c != pack_nibbles(rc)).sum()} code bytes differ"
 
 
+@pytest.mark.parametrize("fmt", W4)
+@pytest.mark.parametrize("shift", [0, 120, 135])
+def test_activation_quantizer_every_bf16_value(fmt, shift):
+    # every finite bf16 bit pattern once, each block of 16 / 32 consecutive
+    # patterns a block of x (rolled by `shift` so that the blocks mix
+    # magnitudes differently); the NVFP4 codes come from a quotient formed
+    # without dividing and must match the exact one
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = np.where((bits & 0x7F80) != 0x7F80, bits, 0).astype(np.uint16)
+    bits = np.roll(bits, shift * 97)
+    x = torch.from_numpy(bits.view(np.int16).reshape(256, 256).copy()).view(torch.bfloat16)
+    if fmt == "w4a4_nvfp4":
+        x = x.float().clamp(-1e30, 1e30).to(torch.bfloat16)   # keep amax / 2688 an ordinary fp32 scale
+    xv = bf16_values(x)
+    c, s, g = _quantize(fmt, x)
+    if fmt == "w4a4_mxfp4":
+        rc, rs = L.quantize_act_mxfp4(xv)
+    else:
+        rc, rs, rg = L.quantize_act_nvfp4(xv)
+        assert np.float32(g) == np.float32(rg)
+    assert np.array_equal(s, rs), f"{(s != rs).sum()} scale codes differ"
+    assert np.array_equal(c, pack_nibbles(rc)), f"{(c != pack_nibbles(rc)).sum()} code bytes differ"
+
+
 def test_nvfp4_activation_quantizer_zero_tensor_and_repeat_calls():
     # an all-zero x takes g_x = 1; the amax reduction's ticket is left at zero
     # by every call, so a second, different call is exact too

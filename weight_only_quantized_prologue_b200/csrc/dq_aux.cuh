@@ -239,25 +239,51 @@ __device__ __forceinline__ uint32_t e2m1x2_mag(float a, float b) {
   return r;
 }
 
-// The codes of one word of two bf16 values (low half at k): each value
-// times `mul` (MXFP4: the block's 2^-e, a product exact in fp32) or divided
-// by `div` (NVFP4: the block's dec(sb) * g, IEEE division), rounded to E2M1,
-// the sign bit of the input kept (so -0 gives code 8, as the packer's codec
-// does).  Returns the byte of the two codes.
-template <bool MX>
-__device__ __forceinline__ uint32_t e2m1_pair(uint32_t w, float f) {
+// f32(v / d), correctly rounded, for the E2M1 rounding that follows (v >= 0,
+// r = f32(1 / d) correctly rounded and normal): Markstein's correction step,
+// as e4m3_quotient.  Below 2^-4 every E2M1 code is 0 and from 8 on it is 6,
+// whatever the quotient's last bits, so q0 is used as it is there.
+__device__ __forceinline__ float e2m1_quotient(float v, float d, float r) {
+  const float q0 = __fmul_rn(v, r);
+  if (!(q0 >= 0x1p-4f && q0 < 8.f)) return q0;
+  return __fmaf_rn(__fmaf_rn(-q0, d, v), r, q0);
+}
+
+// The codes of one word of two bf16 values (low half at k), the sign bit of
+// the input kept (so -0 gives code 8, as the packer's codec does); returns
+// the byte of the two codes.  DIV = 0: each magnitude times f (MXFP4: the
+// block's 2^-e, a product exact in fp32); 1: divided by f (NVFP4: the
+// block's dec(sb) * g) through e2m1_quotient with r = f32(1 / f); 2: by the
+// IEEE division.
+template <int DIV>
+__device__ __forceinline__ uint32_t e2m1_pair(uint32_t w, float f, float r) {
   const float lo = __uint_as_float((w & 0x7FFFu) << 16), hi = __uint_as_float(w & 0x7FFF0000u);
-  const uint32_t mag = MX ? e2m1x2_mag(__fmul_rn(lo, f), __fmul_rn(hi, f))
-                          : e2m1x2_mag(__fdiv_rn(lo, f), __fdiv_rn(hi, f));
+  const uint32_t mag = DIV == 0 ? e2m1x2_mag(__fmul_rn(lo, f), __fmul_rn(hi, f))
+                     : DIV == 1 ? e2m1x2_mag(e2m1_quotient(lo, f, r), e2m1_quotient(hi, f, r))
+                                : e2m1x2_mag(__fdiv_rn(lo, f), __fdiv_rn(hi, f));
   return mag | ((w >> 12) & 0x8u) | ((w >> 24) & 0x80u);
+}
+
+// the codes of a block's words (WB / 4 packed words of 8 codes)
+template <int DIV, int WB>
+__device__ __forceinline__ void e2m1_block(const uint32_t (&w)[WB], float f, float r, uint32_t* packed) {
+#pragma unroll
+  for (int q = 0; q < WB / 4; ++q) {
+    uint32_t pk = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pk |= e2m1_pair<DIV>(w[4 * q + e], f, r) << (8 * e);
+    packed[q] = pk;
+  }
 }
 
 template <bool MX>
 __global__ void __launch_bounds__(256) w4a4_act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
                                                              int rows, int kp, int bn, const float* gx,
                                                              uint8_t* codes, uint32_t* sfw, uint8_t* scales) {
-  pdl_wait();   // x may be the previous grid's output, and that grid may still read the workspace
+  // (the GEMM after this kernel may start now and stream its weights; it
+  // reads what this kernel writes only after waiting for it to complete)
   pdl_launch_dependents();
+  pdl_wait();   // x may be the previous grid's output, and that grid may still read the workspace
   constexpr int VS = MX ? 32 : 16;   // elements per block
   constexpr int WB = VS / 2;         // bf16x2 words per block
   const float g = MX ? 1.f : *reinterpret_cast<const volatile float*>(gx);
@@ -309,14 +335,18 @@ __global__ void __launch_bounds__(256) w4a4_act_quant_kernel(const __nv_bfloat16
         live = f > 0.f;
       }
       word |= sc << (8 * b);
+      uint32_t* pb = packed + b * (WB / 4);
+      if (!live) {
 #pragma unroll
-      for (int q = 0; q < WB / 4; ++q) {
-        uint32_t pk = 0;
-        if (live) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) pk |= e2m1_pair<MX>(w[4 * q + e], f) << (8 * e);
-        }
-        packed[b * (WB / 4) + q] = pk;
+        for (int q = 0; q < WB / 4; ++q) pb[q] = 0u;
+      } else if constexpr (MX) {
+        e2m1_block<0>(w, f, 0.f, pb);
+      } else {
+        const float r = __frcp_rn(f);
+        if (e4m3_quotient_ok(r))
+          e2m1_block<1>(w, f, r, pb);
+        else
+          e2m1_block<2>(w, f, r, pb);
       }
       if (!sfw && row < M && kb < K) scales[(size_t)row * (K / VS) + kb / VS] = (uint8_t)sc;
     }
@@ -339,8 +369,8 @@ __global__ void __launch_bounds__(256) w4a4_act_quant_kernel(const __nv_bfloat16
 constexpr int kActAmaxBlocks = 1024;
 __global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ x, long long count,
                                                        float* partials, unsigned int* ticket, float* gx) {
+  pdl_launch_dependents();   // (the kernels after it wait for its completion before reading what it writes)
   pdl_wait();
-  pdl_launch_dependents();
   float a = 0.f;
   const long long vecs = count / 8;
   const uint4* xv = reinterpret_cast<const uint4*>(x);
