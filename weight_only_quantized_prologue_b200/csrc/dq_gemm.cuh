@@ -147,12 +147,16 @@ struct GemmCfg {
   // takes the rest, up to 8)
   static constexpr int TSA_WST = BN <= 16 ? 3 : 2;
   static constexpr int TSA_XST = (AVAIL - TSA_WST * W_SLOT - (BN <= 32 ? 4 : 2) * Q_SLOT) / (X_SLOT > 0 ? X_SLOT : 1);
-  static constexpr int XST = TSA ? (TSA_XST > 8 ? 8 : TSA_XST < 2 ? 2 : TSA_XST)
+  // (W4A4 at 256-row tiles: 3 x and 5 weight slots, the fastest of the
+  // splits 5/2, 4/3, 3/5 and 2/8 measured at 4096 x 4096 x 4096)
+  static constexpr bool W4WIDE = W4A4 && BN == 256;
+  static constexpr int XST = W4WIDE ? 3
+                             : TSA ? (TSA_XST > 8 ? 8 : TSA_XST < 2 ? 2 : TSA_XST)
                              : (AVAIL - 6 * X_SLOT >= 3 * W_SLOT) ? 6
                              : (AVAIL - 4 * X_SLOT >= 3 * W_SLOT) ? 4
                              : (AVAIL - 3 * X_SLOT >= 3 * W_SLOT) ? 3
                                                                   : 2;
-  static constexpr int WST_RAW = TSA ? TSA_WST : (AVAIL - XST * X_SLOT) / W_SLOT;
+  static constexpr int WST_RAW = W4WIDE ? 5 : TSA ? TSA_WST : (AVAIL - XST * X_SLOT) / W_SLOT;
   static constexpr int WST = WST_RAW < 2 ? 2 : (WST_RAW > 8 ? 8 : WST_RAW);
   static constexpr int QST_RAW = TSA ? (AVAIL - XST * X_SLOT - WST * W_SLOT) / Q_SLOT : 0;
   static constexpr int QST = QST_RAW > 8 ? 8 : QST_RAW;
@@ -311,7 +315,14 @@ __device__ __forceinline__ void prologue_stage(const uint8_t* chunk, int r, int 
 // not evaluated alongside)
 template <int BN, int NT, bool FAST>
 __device__ __forceinline__ void quantize_x_tile_loop(const uint8_t* xs, uint8_t* qs, float s_x, float r_x, int tid) {
-  for (int c = tid; c < BN * 8; c += NT) {
+  // BN * 8 chunks of 16 codes; a compile-time count per thread, unrolled so
+  // that a thread's chunks interleave (a few quantizing warps per SM
+  // sub-partition leave issue slots to fill)
+  constexpr int PER = (BN * 8 + NT - 1) / NT;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int c = tid + i * NT;
+    if (BN * 8 % NT != 0 && c >= BN * 8) break;
     const int row = c >> 3, cc = c & 7;
     const uint8_t* box = xs + (cc >> 2) * BN * 128 + row * 128;
     const uint4 a = lds128(box + (((2 * (cc & 3)) ^ (row & 7)) << 4));
