@@ -190,7 +190,11 @@ struct GemmCfg {
   static constexpr int A_COLS = A_STAGES * (W4A4 ? SF_SLOT : TSA ? STAGE_K / 4 : STAGE_K / 2);
   static constexpr int ACC_COL = A_COLS;
   static constexpr int ACC2_COL = ACC_COL + ISSUERS * BN;   // MLP: layer 2's accumulators
-  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN);
+  // two accumulators where TMEM has room (static FP8 on e4m3 codes at 256-row
+  // tiles: no A operand or scale slots in TMEM): the MMAs of a CTA's next
+  // tile run while the epilogue reads the last one
+  static constexpr int ACC_BUFS = (XQ && STATIC && BN == 256) ? 2 : 1;
+  static constexpr int TMEM_COLS = pow2_at_least(A_COLS + (MLP ? 2 : ACC_BUFS) * ISSUERS * BN);
   static constexpr int BAR_OFF = B2_OFF + B2_BYTES;
   static constexpr int BAR_BYTES = 8 * 80;
   // each epilogue thread's row factor and bias, parked in shared memory over
@@ -202,7 +206,7 @@ struct GemmCfg {
   // warp 0 weight producer, 1 and 10 MMA issuers, 2..9 prologue/epilogue,
   // 11 x producer
   static constexpr int THREADS = 384;
-  static_assert(A_COLS + (MLP ? 2 : 1) * ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
+  static_assert(A_COLS + (MLP ? 2 : ACC_BUFS) * ISSUERS * BN <= (BN <= 64 ? 256 : 512), "TMEM budget");
   static_assert(!(MLP && BN > 64), "the MLP runs x tiles of at most 64 rows");
   static_assert(!(STATIC && !XQ && BN > 128), "the fused static-FP8 tile holds at most 128 x rows");
   static_assert(!(W4A4 && BN < 32), "W4A4 x tiles hold 32 rows or more (one scale column per 32 rows)");
@@ -380,7 +384,9 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
   uint64_t* acc2_full = b2ready + 1;      // MLP: layer 2's accumulators complete
   uint64_t* xready = acc2_full + 1;       // [8] fused static with A in TMEM: operand slot written
   uint64_t* qempty = xready + 8;          // [8]   ... and read by the MMAs
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 8);
+  uint64_t* acc_full_b[2] = {acc_full, qempty + 8};        // the second accumulator's, if any
+  uint64_t* acc_empty_b[2] = {acc_empty, qempty + 9};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* recv = reinterpret_cast<float*>(smem + C::RECV_OFF);             // [S][128][BN/S]
   uint32_t* rflag = reinterpret_cast<uint32_t*>(smem + C::RFLAG_OFF);     // [S][4]: sender rank, row quadrant
@@ -405,6 +411,8 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     }
     mbar_init(acc_full, C::ISSUERS);
     mbar_init(acc_empty, 8);
+    mbar_init(acc_full_b[1], C::ISSUERS);
+    mbar_init(acc_empty_b[1], 8);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(recv_bar, 1);
@@ -517,12 +525,14 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     if (lane == 0 && (warp == 1 || C::ISSUERS == 2)) {
       const int which = warp == 1 ? 0 : 1;   // k-steps [which*KK, (which+1)*KK) of each stage
       constexpr int KK = C::KK;
-      const uint32_t d_tmem = tmem + C::ACC_COL + which * BN;
       int ws = 0, xs = 0, as = 0;
       uint32_t wph = 0, xph = 0, aph = 0;
       bool ok = true, issued = false;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
-        if (!mbar_wait(acc_empty, (t & 1) ^ 1, ctl())) break;
+        const int ab = C::ACC_BUFS == 2 ? (t & 1) : 0;              // this tile's accumulator
+        const uint32_t acc_ph = (uint32_t)(C::ACC_BUFS == 2 ? (t >> 1) : t) & 1u;
+        const uint32_t d_tmem = tmem + C::ACC_COL + ab * (C::ISSUERS * BN) + which * BN;
+        if (!mbar_wait(acc_empty_b[ab], acc_ph ^ 1, ctl())) break;
         tc_fence_after();
         for (int j = 0; j < nst; ++j) {
           const uint32_t xb = smem_u32(x_ring + xs * C::X_SLOT);
@@ -587,7 +597,10 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
               aph ^= 1;
             }
           } else {
-            if (!mbar_wait(&full_w[ws], wph, ctl()) || !mbar_wait(&aready[xs], xph, ctl())) { ok = false; break; }
+            // (x quantized in the kernel: the prologue warps signal each x
+            // slot's e4m3 operand; quantized beforehand: the x copy itself)
+            if (!mbar_wait(&full_w[ws], wph, ctl()) ||
+                !mbar_wait(C::XQ ? &full_x[xs] : &aready[xs], xph, ctl())) { ok = false; break; }
             tc_fence_after();
             const uint32_t wb = smem_u32(w_ring + ws * C::W_SLOT) + which * KK * 32;
             const uint32_t qb = xb + C::Q_OFF + which * KK * 32;
@@ -617,7 +630,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit(acc_full_b[ab]);
       }
       if constexpr (C::MLP) {
         // layer 2 on this CTA's k-slice: A = layer 2's weight chunk, B = the
@@ -830,51 +843,67 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       } else {
         // static FP8: quantize each x tile into the e4m3 half of its slot
         // (the slot was refilled only after its previous MMAs completed);
-        // pre-quantized x is only passed on
-        for (int j = 0; j < nst; ++j) {
-          if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
-          if constexpr (!C::XQ) {
+        // pre-quantized x needs nothing here (the MMAs wait for its copy)
+        if constexpr (!C::XQ) {
+          for (int j = 0; j < nst; ++j) {
+            if (!mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
             uint8_t* xd = x_ring + xs * C::X_SLOT;
             quantize_x_tile<BN>(xd, xd + C::Q_OFF, p.s_x, p.r_x, et);
             fence_proxy_async_smem();
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&aready[xs]);
-          if (++xs == C::XST) {
-            xs = 0;
-            xph ^= 1;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&aready[xs]);
+            if (++xs == C::XST) {
+              xs = 0;
+              xph ^= 1;
+            }
           }
         }
       }
       if (!ok) break;
       // ---- epilogue of this tile
-      if (!mbar_wait_warp(acc_full, t & 1, ctl())) { ok = false; break; }
+      const int ab = C::ACC_BUFS == 2 ? (t & 1) : 0;                  // its accumulator
+      const uint32_t acc_ph = (uint32_t)(C::ACC_BUFS == 2 ? (t >> 1) : t) & 1u;
+      if (!mbar_wait_warp(acc_full_b[ab], acc_ph, ctl())) { ok = false; break; }
       tc_fence_after();
       if constexpr (CHUNKED) {
-        // one accumulator (one issuer): 32 columns at a time, the TMEM
-        // accumulator released after the last load, then that chunk stored
+        // one accumulator (one issuer): the thread's 128 columns read 32 at
+        // a time and kept as finished outputs (bf16 pairs, or e4m3 quads),
+        // the accumulator released after the last read, then everything
+        // stored (so the stores overlap the next tile's MMAs)
         const int n_row = (tile / p.m_tiles) * TILE_N + r, m_tile = tile % p.m_tiles;
         const float e_sig = epi[et], e_bias = epi[256 + et];
-#pragma unroll 1
+        constexpr int PW = QOUT ? HALF / 4 : HALF / 2;   // packed words of outputs
+        uint32_t pk[PW];
+#pragma unroll
         for (int c32 = 0; c32 < HALF / 32; ++c32) {
           float a[32];
-          tmem_ld32(tmem + lane_base + C::ACC_COL + h * HALF + c32 * 32, a);
+          tmem_ld32(tmem + lane_base + C::ACC_COL + ab * BN + h * HALF + c32 * 32, a);
           tmem_wait_ld();
-          if (c32 == HALF / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-          }
-          if (n_row < p.N) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int m = m_tile * BN + h * HALF + c32 * 32 + i;
-              if (m < p.M) {
-                if constexpr (!QOUT)
-                  p.y[(size_t)m * p.N + n_row] = __float2bfloat16_rn(fmaf(a[i], e_sig, e_bias));
-                else
-                  p.yq[(size_t)m * p.N + n_row] = out_code(p, fmaf(a[i], e_sig, e_bias));
-              }
+          for (int i = 0; i < 32; i += (QOUT ? 4 : 2)) {
+            if constexpr (!QOUT) {
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(fmaf(a[i], e_sig, e_bias), fmaf(a[i + 1], e_sig, e_bias));
+              pk[(c32 * 32 + i) / 2] = *reinterpret_cast<const uint32_t*>(&v2);
+            } else {
+              uint32_t w = 0;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) w |= (uint32_t)out_code(p, fmaf(a[i + k], e_sig, e_bias)) << (8 * k);
+              pk[(c32 * 32 + i) / 4] = w;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty_b[ab]);
+        if (n_row < p.N) {
+#pragma unroll
+          for (int i = 0; i < HALF; ++i) {
+            const int m = m_tile * BN + h * HALF + i;
+            if (m < p.M) {
+              if constexpr (!QOUT)
+                p.y[(size_t)m * p.N + n_row] = __ushort_as_bfloat16((unsigned short)(pk[i / 2] >> (16 * (i & 1))));
+              else
+                p.yq[(size_t)m * p.N + n_row] = (uint8_t)(pk[i / 4] >> (8 * (i & 3)));
             }
           }
         }
