@@ -79,3 +79,59 @@ def test_sweep_shapes_match_oracle(fmt, M, K, N, rows):
         check_close(yv[sel], ref, x_eff, wdq)
     finally:
         dq.dqgemm_destroy(h)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "fp8", "fp8_static", "w4a4_mxfp4"])
+@pytest.mark.parametrize("M", [1, 32])
+def test_skinny_tiles_more_than_sms(fmt, M):
+    # 160 output tiles (N = 20480) at 1 and 32 rows: more tiles than SMs, so
+    # the skinny tile is kept and CTAs loop over whole tiles (persistent);
+    # with 74..148 tiles the plan takes the 128-row tile instead
+    from gpu_util import base_fmt, make_layer, w4a4_effective_x
+
+    K, N = 512, 20480
+    x, w, b = synthetic.linear_inputs(M, K, N, seed=M + 5)
+    xv = bf16_values(x)
+    s_x = L.act_scale(xv.min(), xv.max())
+    h, st, wdq = make_layer(fmt, w.numpy().astype(np.float64), None if fmt == "fp8_static" else b.cuda(),
+                            act_scale=s_x)
+    try:
+        plan = dq.dqgemm_get_plan(h, M)
+        assert plan["bn"] == (32 if fmt.startswith("w4a4") or M == 32 else 16), plan
+        assert plan["max_segments"] == 1 and plan["n_tiles"] > plan["grid"], plan
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dq.dqgemm_run(h, x.cuda(), M, y)
+        torch.cuda.synchronize()
+        assert dq.dqgemm_last_error(h) == 0
+        bias = None if fmt == "fp8_static" else bf16_values(b)
+        if fmt.startswith("w4a4"):
+            x_eff = w4a4_effective_x(fmt, xv)
+            ref = L.w4a4_linear_ref(base_fmt(fmt), xv, st["packed"], st["scales"], st["global_scale"], bias)
+        else:
+            x_eff = static_effective_x(xv, s_x) if fmt == "fp8_static" else xv
+            ref = L.linear_ref(x_eff, wdq, bias)
+        check_close(bf16_values(y), ref, x_eff, wdq)
+    finally:
+        dq.dqgemm_destroy(h)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "fp8"])
+def test_skinny_rows_take_the_128_row_tile_when_tiles_fill_the_gpu(fmt):
+    # 112 output tiles (N = 14336): the K range cannot be split, so one CTA
+    # per SM streams a whole tile, on the 128-row tile
+    from gpu_util import make_layer
+
+    K, N, M = 512, 14336, 24
+    x, w, b = synthetic.linear_inputs(M, K, N, seed=9)
+    h, st, wdq = make_layer(fmt, w.numpy().astype(np.float64), b.cuda())
+    try:
+        plan = dq.dqgemm_get_plan(h, M)
+        assert plan["bn"] == 128 and plan["max_segments"] == 1 and plan["grid"] == 112, plan
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        dq.dqgemm_run(h, x.cuda(), M, y)
+        torch.cuda.synchronize()
+        assert dq.dqgemm_last_error(h) == 0
+        xv = bf16_values(x)
+        check_close(bf16_values(y), L.linear_ref(xv, wdq, bf16_values(b)), xv, wdq)
+    finally:
+        dq.dqgemm_destroy(h)

@@ -451,6 +451,18 @@ int cluster_capacity(dqgemm_s* h, int bn, int split) {
 int pick_bn(const dqgemm_s* h, int M, bool xq) {
   int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   if (is_w4a4(h->fmt) && bn < 32) bn = 32;   // one block-scale column per 32 x rows
+  // From 16 to 64 rows, when the output tiles fill more than half the SMs
+  // (so the K range cannot be split) and fit one wave, every CTA streams a
+  // whole tile alone on its SM: the 128-row tile's larger rings serve it
+  // better than the skinny tiles' two-CTAs-per-SM budget (measured at
+  // 4096 x 14336: INT4 24.0 against 29.6 us, FP8-WO 21.7 against 27.0).
+  // Not below 16 rows, where x boxes of 128 rows with 8 or fewer rows in the
+  // tensor ran twice as slow (W4A4 is exempt: its quantized x is padded to
+  // the tile), and not for fused static FP8, whose 128-row tile keeps few
+  // x slots (54 against 23 us).
+  if (bn <= 64 && (M >= 16 || is_w4a4(h->fmt)) && !(h->fmt == FMT_FP8S && !xq) &&
+      2 * (long long)h->n_tiles > h->num_sms && h->n_tiles <= h->num_sms)
+    bn = 128;
   if (M > 128 && !(h->fmt == FMT_FP8S && !xq)) {
     const long long sms = h->num_sms, nt = h->n_tiles;
     const long long t256 = (M + 255) / 256 * nt, t128 = (M + 127) / 128 * nt;
