@@ -126,3 +126,26 @@ def test_quantizer_codes_exact_next_to_e4m3_midpoints(s_x):
             assert not bad.any(), f"M={M}: {bad.sum()} outputs off by more than bf16 rounding"
         finally:
             dq.dqgemm_destroy(h)
+
+
+def test_quantized_linear_prequantizes_earlier_when_tiles_fill_the_gpu():
+    # N = 14336 (112 output tiles): from 16 rows the layer quantizes x once
+    # and runs the FP8 GEMM on codes, planned on the 128-row tile; same
+    # result as the fused kernel, and the oracle's
+    M, K, N = 24, 512, 14336
+    x, W, _ = synthetic.linear_inputs(M, K, N, seed=8)
+    xc = x.cuda()
+    xv = bf16_values(x)
+    s_x = L.act_scale(xv.min(), xv.max())
+    lin = dq.QuantizedLinear.from_float("fp8_static", W.cuda(), None, act_scale=s_x)
+    try:
+        assert lin._static_prequant_m == lin.STATIC_PREQUANT_M_WIDE <= M < lin.STATIC_PREQUANT_M
+        y = lin(xc)
+        y_fused = run(lin.handle, xc, N)
+        assert torch.equal(y.view(torch.int16), y_fused.view(torch.int16))
+        st = L.quantize_pack("fp8", W.numpy().astype(np.float64))
+        wdq = L.dequant_exact("fp8", st["packed"], st["scales"])
+        x_eff = static_effective_x(xv, s_x)
+        check_close(bf16_values(y), L.linear_ref(x_eff, wdq), x_eff, wdq)
+    finally:
+        lin.close()

@@ -102,8 +102,14 @@ class QuantizedLinear:
     library, so the caller may drop them afterwards."""
 
     # static FP8 from this many rows on: quantize x once, then the FP8 GEMM
-    # (the fused kernel re-quantizes x for every 128-channel tile)
+    # (the fused kernel re-quantizes x for every 128-channel tile) ...
     STATIC_PREQUANT_M = 128
+    # ... and from this many when the output tiles fill more than half the
+    # SMs in one wave: the GEMM on codes then takes the 128-row tile, one CTA
+    # per SM over the whole K range, which the fused kernel does not (at
+    # 4096 x 14336: 19.6 against 33.6 us at 32 rows; up to 16 rows the fused
+    # 16-row tile is faster, 23.2 against 25.5)
+    STATIC_PREQUANT_M_WIDE = 17
 
     def __init__(self, fmt, K, N, packed, scales, global_scale=1.0, bias=None):
         import torch
@@ -117,6 +123,10 @@ class QuantizedLinear:
         if bias is not None:
             _require(bias, "bias", shape=(N,), dtype=torch.bfloat16, device=packed.device)
         self.fmt, self.K, self.N = fmt, K, N
+        sms = torch.cuda.get_device_properties(packed.device).multi_processor_count
+        n_tiles = (N + 127) // 128
+        self._static_prequant_m = (self.STATIC_PREQUANT_M_WIDE if 2 * n_tiles > sms and n_tiles <= sms
+                                   else self.STATIC_PREQUANT_M)
         self.device = packed.device               # the handle belongs to this device
         # with one visible GPU the current device can only be this one
         self._check_current = torch.cuda.device_count() > 1
@@ -173,7 +183,7 @@ class QuantizedLinear:
         out = self._out(out, M, torch.bfloat16, x.device)
         if M == 0:
             return out
-        if self.fmt == "fp8_static" and M >= self.STATIC_PREQUANT_M:
+        if self.fmt == "fp8_static" and M >= self._static_prequant_m:
             q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
             dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
             dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)
@@ -190,7 +200,7 @@ class QuantizedLinear:
         out = self._out(out, M, torch.uint8, x.device)
         if M == 0:
             return out
-        if self.fmt == "fp8_static" and M >= self.STATIC_PREQUANT_M:
+        if self.fmt == "fp8_static" and M >= self._static_prequant_m:
             q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
             dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
             dqgemm_run_fp8_static_quantized_out(self._h, q, M, out, s_out, stream)
