@@ -2,7 +2,7 @@
 //
 // y[M, N] = x[M, K] . deq(W)^T + b, computed as y^T = deq(W) . x^T so that
 // the 128 weight rows of a tile are the tcgen05 MMA's M and the activation
-// rows are its N (BN = 16..128): the skinny decode shapes the quantized-Linear
+// rows are its N (BN = 16..256): the skinny decode shapes the quantized-Linear
 // pages run (x of 32 rows) keep the tensor core busy on the weight side.
 //
 // CTA = 12 warps, warp-specialized:
@@ -10,24 +10,33 @@
 //               weight chunk per stage into a ring of up to 8 slots, from
 //               CTA entry on (weights never depend on the previous grid)
 //   warp 11     x producer: after the grid-dependency wait, the TMA box
-//               load(s) of the stage's x tile into a 2-3 slot ring
+//               load(s) of the stage's x tile (bf16, or codes quantized
+//               beforehand, plus W4A4's scale words) into the x ring
 //   warps 1, 10 MMA issuers: one thread each issues tcgen05.mma for half of
-//               every stage's k-steps into its own TMEM accumulator (a single
-//               thread issues only one MMA every ~80 cycles) and commits the
-//               slot / operand / accumulator barriers
-//   warps 2..9  the prologue: unpack + scale the packed codes of one weight
-//               row per thread (two threads per row, one per k-half) into
-//               bf16 operands written straight to TMEM (the MMA reads A from
-//               TMEM), or, for static FP8, quantize the x tile to e4m3 into
-//               shared memory; then the epilogue (tcgen05.ld of both
-//               accumulators, scale, bias, bf16 cast, store).
+//               every stage's k-steps into its own TMEM accumulator (one
+//               issuer at 256-row tiles) and commits the slot / operand /
+//               accumulator barriers
+//   warps 2..9  the prologue, then the epilogue:
+//               - weight-only formats: unpack + scale the packed codes of one
+//                 weight row per thread (two threads per row, one per
+//                 k-half) into bf16 operands written straight to TMEM (the
+//                 MMA reads A from TMEM);
+//               - fused static FP8: warps 2..5 copy the e4m3 weight rows into
+//                 TMEM (the FP8 MMA reads A there) and warps 6..9 quantize
+//                 the bf16 x tile to e4m3 operands in shared memory;
+//               - W4A4: write each stage's block scales of both operands into
+//                 TMEM (the MMA reads both operands from shared memory);
+//               - static FP8 on codes: nothing (both operands in shared
+//                 memory; its 256-row tiles double-buffer the accumulator,
+//                 so these warps' epilogue overlaps the next tile);
+//               then tcgen05.ld of the accumulator(s), scale, bias, cast,
+//               store.
 // Work split: a tile of 128 output channels x BN activation rows is either
 // computed whole by one CTA (persistent loop over tiles), or its K range is
-// split over the S CTAs of a thread-block cluster: each writes its fp32
-// partial tile into its own shared memory and, after a cluster barrier, rank
-// q reads its share of the columns from all S partials over distributed
-// shared memory and adds them in rank order (deterministic, no global
-// scratch).
+// split over the S CTAs of a thread-block cluster: each sends every peer its
+// partial of the peer's columns into the peer's shared memory (st.async),
+// and each adds the S partials of its own columns in rank order
+// (deterministic, no global scratch).
 // Back-to-back calls overlap through programmatic dependent launch: a CTA
 // sets up and starts streaming its (read-only) weights before waiting for the
 // previous grid; it reads x and writes y only after that wait.
