@@ -684,6 +684,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     int tile = 0;
     int ws = 0, xs = 0, as = 0, qs = 0;     // ring positions, kept across the tiles of a persistent CTA
     uint32_t wph = 0, xph = 0, aph = 0, qph = 0;
+    int pre = 0;                            // stages of this tile already handled (prefilled during the last)
     bool ok = true, have_acc = false;
     for (int t = 0; ok && t < wk.ntiles; ++t) {
       tile = wk.first_tile + t * wk.tile_step;
@@ -711,8 +712,8 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         // the k-steps t = 2h, 2h + 1 into its own quadrant, from the weight
         // chunk's and the x slot's scale words ([t][row] each)
         constexpr int NB = BN / 32;
-        for (int j = 0; j < nst; ++j) {
-          if (!mbar_wait_warp(&full_w[ws], wph, ctl()) || !mbar_wait_warp(&full_x[xs], xph, ctl())) { ok = false; break; }
+        const auto sf_stage = [&]() -> bool {
+          if (!mbar_wait_warp(&full_w[ws], wph, ctl()) || !mbar_wait_warp(&full_x[xs], xph, ctl())) return false;
           const uint32_t* wsf = reinterpret_cast<const uint32_t*>(w_ring + ws * C::W_SLOT + W4_SF_OFF);
           const uint32_t* xsf = reinterpret_cast<const uint32_t*>(x_ring + xs * C::X_SLOT + C::XSF_OFF);
           uint32_t va[8], vb[2 * NB];
@@ -724,7 +725,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
 #pragma unroll
             for (int c = 0; c < NB; ++c) vb[u * NB + c] = xsf[t * BN + c * 32 + lane];
           }
-          if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) { ok = false; break; }
+          if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) return false;
           tc_fence_after();
           const uint32_t ts = tmem + lane_base + as * C::SF_SLOT;
           tmem_st_cols<8>(ts + 8 * h, va);
@@ -746,6 +747,17 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
             as = 0;
             aph ^= 1;
           }
+          return true;
+        };
+        // this tile's stages not handled yet, then the next tile's first
+        // ones (their TMEM slots free up as this tile's MMAs complete), so
+        // that its MMAs can start as soon as the accumulator is read
+        for (int j = pre; j < nst; ++j)
+          if (!sf_stage()) { ok = false; break; }
+        pre = 0;
+        if (ok && t + 1 < wk.ntiles) {
+          for (int j = 0; j < (nst < C::A_STAGES ? nst : C::A_STAGES); ++j, ++pre)
+            if (!sf_stage()) { ok = false; break; }
         }
       } else if constexpr (C::TSA) {
         if (h == 0) {
@@ -820,8 +832,8 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
       } else if constexpr (!C::STATIC) {
         // the weight operand needs no x: the first A_STAGES stages are
         // unpacked before the grid-dependency wait has even returned
-        for (int j = 0; j < nst; ++j) {
-          if (!mbar_wait_warp(&full_w[ws], wph, ctl())) { ok = false; break; }
+        const auto unpack_stage = [&]() -> bool {
+          if (!mbar_wait_warp(&full_w[ws], wph, ctl())) return false;
           // unpack the first half while the TMEM slot may still be read by
           // the MMAs of an earlier stage, then store it, unpack the second
           // half (after which the weight slot is free) and store it
@@ -829,7 +841,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           const uint32_t ta = tmem + lane_base + as * (STAGE_K / 2) + h * 32;
           uint32_t o[16];
           prologue_half<FMT>(chunk, r, h, 0, p.mx_bias, o);
-          if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) { ok = false; break; }
+          if (!mbar_wait_warp(&aempty[as], aph ^ 1, ctl())) return false;
           tc_fence_after();
           tmem_st16(ta, o);
           prologue_half<FMT>(chunk, r, h, 1, p.mx_bias, o);
@@ -848,6 +860,17 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
             as = 0;
             aph ^= 1;
           }
+          return true;
+        };
+        // this tile's stages not unpacked yet, then the next tile's first
+        // ones (their TMEM slots free up as this tile's MMAs complete), so
+        // that its MMAs can start as soon as the accumulator is read
+        for (int j = pre; j < nst; ++j)
+          if (!unpack_stage()) { ok = false; break; }
+        pre = 0;
+        if (ok && t + 1 < wk.ntiles) {
+          for (int j = 0; j < (nst < C::A_STAGES ? nst : C::A_STAGES); ++j, ++pre)
+            if (!unpack_stage()) { ok = false; break; }
         }
       } else {
         // static FP8: quantize each x tile into the e4m3 half of its slot
