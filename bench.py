@@ -840,6 +840,9 @@ def run_sweep(args):
                     t1.record(stream)
                     t1.synchronize()
                 us = t0.elapsed_time(t1) * 1000.0 / reps
+                for l in layers:
+                    # a timed-out call wrote nothing: its time is no measurement
+                    assert l.last_error() == 0, f"device-side wait timed out: {fmt} {M}x{K}x{N}"
                 byts = algorithmic_bytes(fmt, M, K, N, bias=fmt != "fp8_static")
                 gbs = byts / (us * 1e-6) / 1e9
                 tflops = flops / (us * 1e-6) / 1e12

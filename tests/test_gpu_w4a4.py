@@ -148,6 +148,9 @@ def _check_gemm(fmt, M, K, N, seed, bias, layer=None):
     (300, 1024, 1024, True, 128, 4),     # three m-tiles
     (1024, 512, 2560, True, 256, 1),     # 256-row tiles, whole tiles over the SMs
     (768, 256, 6400, False, 128, 1),     # 300 128-row tiles: two or three per CTA
+    (2048, 1024, 4736, True, 256, 1),    # 296 256-row tiles of 4 stages (more than the x slots), two per
+                                         # CTA: a CTA prepares its next tile's first stages while its
+                                         # rings still hold this tile's
 ])
 def test_gemm_matches_oracle(fmt, M, K, N, bias, bn, split):
     plan = _check_gemm(fmt, M, K, N, seed=M + K + N, bias=bias)

@@ -195,8 +195,20 @@ struct GemmCfg {
   static constexpr int SFB_OFF = 16;   // within a scale slot
   // (TSA: every TMEM column the accumulators leave, at most 8 slots)
   static constexpr int TSA_STAGES = ((BN <= 64 ? 256 : 512) - 2 * BN) / 32 > 8 ? 8 : ((BN <= 64 ? 256 : 512) - 2 * BN) / 32;
-  static constexpr int A_STAGES = W4A4 ? 3 : TSA ? TSA_STAGES : STATIC ? 0 : (BN == 64 ? 2 : 3);
+  // (W4A4: as many scale slots as the accumulators leave, at most 8; the
+  // scales of a stage pass through the prologue warps, and a deeper ring
+  // keeps more stages of that hand-over in flight)
+  static constexpr int W4_STAGES = ((BN <= 64 ? 256 : 512) - ISSUERS * BN) / SF_SLOT > 8
+                                       ? 8 : ((BN <= 64 ? 256 : 512) - ISSUERS * BN) / SF_SLOT;
+  static constexpr int A_STAGES = W4A4 ? W4_STAGES : TSA ? TSA_STAGES : STATIC ? 0 : (BN == 64 ? 2 : 3);
   static constexpr int A_COLS = A_STAGES * (W4A4 ? SF_SLOT : TSA ? STAGE_K / 4 : STAGE_K / 2);
+  // stages of a persistent CTA's next tile the prologue warps may prepare
+  // before this tile's epilogue: at most its TMEM slots, and for W4A4 (whose
+  // weight and x slots only the MMAs free, which wait for that epilogue) at
+  // most the weight and x slots too, else the preparation would wait on
+  // itself
+  static constexpr int PREFILL_RAW = W4A4 ? (XST < WST ? XST : WST) : A_STAGES;
+  static constexpr int PREFILL = PREFILL_RAW < A_STAGES ? PREFILL_RAW : A_STAGES;
   static constexpr int ACC_COL = A_COLS;
   static constexpr int ACC2_COL = ACC_COL + ISSUERS * BN;   // MLP: layer 2's accumulators
   // two accumulators where TMEM has room (static FP8 on e4m3 codes at 256-row
@@ -756,7 +768,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           if (!sf_stage()) { ok = false; break; }
         pre = 0;
         if (ok && t + 1 < wk.ntiles) {
-          for (int j = 0; j < (nst < C::A_STAGES ? nst : C::A_STAGES); ++j, ++pre)
+          for (int j = 0; j < (nst < C::PREFILL ? nst : C::PREFILL); ++j, ++pre)
             if (!sf_stage()) { ok = false; break; }
         }
       } else if constexpr (C::TSA) {
@@ -869,7 +881,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
           if (!unpack_stage()) { ok = false; break; }
         pre = 0;
         if (ok && t + 1 < wk.ntiles) {
-          for (int j = 0; j < (nst < C::A_STAGES ? nst : C::A_STAGES); ++j, ++pre)
+          for (int j = 0; j < (nst < C::PREFILL ? nst : C::PREFILL); ++j, ++pre)
             if (!unpack_stage()) { ok = false; break; }
         }
       } else {
