@@ -11,7 +11,8 @@
 //               CTA entry on (weights never depend on the previous grid)
 //   warp 11     x producer: after the grid-dependency wait, the TMA box
 //               load(s) of the stage's x tile (bf16, or codes quantized
-//               beforehand, plus W4A4's scale words) into the x ring
+//               beforehand, plus W4A4's scale words) into the x ring (a
+//               single-tile CTA's first ring issued by one lane per stage)
 //   warps 1, 10 MMA issuers: one thread each issues tcgen05.mma for half of
 //               every stage's k-steps into its own TMEM accumulator (one
 //               issuer at 256-row tiles) and commits the slot / operand /
@@ -20,7 +21,8 @@
 //               - weight-only formats: unpack + scale the packed codes of one
 //                 weight row per thread (two threads per row, one per
 //                 k-half) into bf16 operands written straight to TMEM (the
-//                 MMA reads A from TMEM);
+//                 MMA reads A from TMEM), taking turns with the CTA of the
+//                 neighbouring call on the same SM (g_sm_turn);
 //               - fused static FP8: warps 2..5 copy the e4m3 weight rows into
 //                 TMEM (the FP8 MMA reads A there) and warps 6..9 quantize
 //                 the bf16 x tile to e4m3 operands in shared memory;
@@ -382,6 +384,57 @@ __device__ __forceinline__ void quantize_x_tile(const uint8_t* xs, uint8_t* qs, 
 // QOUT: the output leaves as the next static-FP8 layer's e4m3 codes (a
 // separate instantiation, so the common bf16 epilogue stays as compact as
 // it can be)
+// Back-to-back skinny calls share each SM: the next call's CTA lands while
+// this call's CTA is still waiting for the previous grid, and after that wait
+// this CTA still has to unpack the stages that did not fit in TMEM before
+// it; two CTAs unpacking at once run at half speed each.  So a single-tile
+// CTA with such stages marks its SM (its grid's tag) from the end of its
+// early unpacks to the end of its late ones, and a CTA of another grid that
+// lands on a marked SM holds its early unpacks (which only have to be done by
+// the time its own wait returns) until the mark clears, or for at most
+// kTurnWaitNs.  The table is a scheduling hint only: a stale or torn entry
+// costs at most that bounded delay, never a result.
+__device__ uint32_t g_sm_turn[256];
+constexpr uint64_t kTurnWaitNs = 6000;
+
+__device__ __forceinline__ uint32_t sm_id() {
+  uint32_t s;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
+  return s & 255u;
+}
+// an odd (so nonzero) tag of this launch
+__device__ __forceinline__ uint32_t grid_tag() {
+  uint64_t g;
+  asm volatile("mov.u64 %0, %%gridid;" : "=l"(g));
+  return (uint32_t)g * 2u + 1u;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+// wait (bounded) until no other grid's CTA holds this SM's mark; false if
+// the wait gave up, after clearing the mark it gave up on (so that a mark
+// left behind delays one CTA, not every later one)
+__device__ __forceinline__ bool sm_turn_wait(uint32_t sm, uint32_t tag) {
+  uint32_t v = ld_relaxed_gpu(&g_sm_turn[sm]);
+  if (v == 0u || v == tag) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(128);
+    const uint32_t w = ld_relaxed_gpu(&g_sm_turn[sm]);
+    if (w == 0u || w == tag) return true;
+    if (w != v) {
+      v = w;   // another CTA took the mark: its own turn starts now
+      continue;
+    }
+    if (globaltimer_ns() - t0 >= kTurnWaitNs) {
+      atomicCAS(&g_sm_turn[sm], v, 0u);
+      return false;
+    }
+  }
+}
+
 template <int FMT, int BN, bool QOUT>
 __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                          const GemmParams p) {
@@ -504,33 +557,49 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     __syncwarp();
   } else if (warp == 11) {
     // ------------------------------------------------------------ x producer
-    if (lane == 0) {
+    // one stage's x copy into slot xs (bf16 boxes, or codes and W4A4's
+    // scale words)
+    const auto issue_x = [&](int xs, int ks, int m_tile) {
+      uint8_t* xd = x_ring + xs * C::X_SLOT;
+      if constexpr (C::XQ) {
+        // codes straight into the operand buffer of the slot (128 bytes
+        // of each row per stage), and for W4A4 the stage's scale words
+        mbar_arrive_expect_tx(&full_x[xs], C::Q_BYTES + C::XSF_BYTES);
+        tma_load_2d(xd + C::Q_OFF, &tmap_x, ks * 128, m_tile * BN, &full_x[xs]);
+        if constexpr (C::W4A4)
+          bulk_g2s(xd + C::XSF_OFF, p.xsf + ((size_t)m_tile * KS + ks) * 4 * BN, C::XSF_BYTES, &full_x[xs]);
+      } else {
+        mbar_arrive_expect_tx(&full_x[xs], C::X_BYTES);
+        if (p.x3d) {
+          tma_load_3d(xd, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[xs]);
+        } else {
+          tma_load_2d(xd, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
+          tma_load_2d(xd + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[xs]);
+        }
+      }
+    };
+    // A single-tile CTA's first ring of x copies is issued by that many
+    // lanes at once (one stage each): on the critical path after the wait,
+    // one thread issuing them in turn took ~0.3 us a copy.  The rest, and
+    // every copy of a persistent CTA, come from lane 0 in ring order.
+    const int nfirst = wk.ntiles == 1 ? (nst < C::XST ? nst : C::XST) : 0;
+    if (lane < nfirst) {
       pdl_wait();   // x may be the previous grid's output
-      int xs = 0, it = 0;
-      uint32_t xph = 0;
+      const int m_tile = wk.first_tile - (wk.first_tile / p.m_tiles) * p.m_tiles;
+      issue_x(lane, wk.kb + lane, m_tile);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      if (nfirst == 0) pdl_wait();
+      int it = nfirst, xs = nfirst == C::XST ? 0 : nfirst;
+      uint32_t xph = nfirst == C::XST ? 1u : 0u;
       bool ok = true;
       for (int t = 0; ok && t < wk.ntiles; ++t) {
         const int tile = wk.first_tile + t * wk.tile_step;
         const int m_tile = tile - (tile / p.m_tiles) * p.m_tiles;
-        for (int ks = wk.kb; ks < wk.ke; ++ks, ++it) {
+        for (int ks = wk.kb + (t == 0 ? nfirst : 0); ks < wk.ke; ++ks, ++it) {
           if (it >= C::XST && !mbar_wait(&xempty[xs], xph ^ 1, ctl())) { ok = false; break; }
-          uint8_t* xd = x_ring + xs * C::X_SLOT;
-          if constexpr (C::XQ) {
-            // codes straight into the operand buffer of the slot (128 bytes
-            // of each row per stage), and for W4A4 the stage's scale words
-            mbar_arrive_expect_tx(&full_x[xs], C::Q_BYTES + C::XSF_BYTES);
-            tma_load_2d(xd + C::Q_OFF, &tmap_x, ks * 128, m_tile * BN, &full_x[xs]);
-            if constexpr (C::W4A4)
-              bulk_g2s(xd + C::XSF_OFF, p.xsf + ((size_t)m_tile * KS + ks) * 4 * BN, C::XSF_BYTES, &full_x[xs]);
-          } else {
-            mbar_arrive_expect_tx(&full_x[xs], C::X_BYTES);
-            if (p.x3d) {
-              tma_load_3d(xd, &tmap_x, 0, m_tile * BN, ks * 2, &full_x[xs]);
-            } else {
-              tma_load_2d(xd, &tmap_x, ks * STAGE_K, m_tile * BN, &full_x[xs]);
-              tma_load_2d(xd + BN * 128, &tmap_x, ks * STAGE_K + 64, m_tile * BN, &full_x[xs]);
-            }
-          }
+          issue_x(xs, ks, m_tile);
           if (++xs == C::XST) {
             xs = 0;
             xph ^= 1;
@@ -698,6 +767,7 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
     uint32_t wph = 0, xph = 0, aph = 0, qph = 0;
     int pre = 0;                            // stages of this tile already handled (prefilled during the last)
     bool ok = true, have_acc = false;
+    bool marked = false;                    // this CTA's mark in g_sm_turn is set (one thread)
     for (int t = 0; ok && t < wk.ntiles; ++t) {
       tile = wk.first_tile + t * wk.tile_step;
       // this row's epilogue factor and bias: read-only, fetched now so the
@@ -876,9 +946,24 @@ __global__ void __launch_bounds__(384, BN <= 64 ? 2 : 1) dq_gemm_kernel(const __
         };
         // this tile's stages not unpacked yet, then the next tile's first
         // ones (their TMEM slots free up as this tile's MMAs complete), so
-        // that its MMAs can start as soon as the accumulator is read
-        for (int j = pre; j < nst; ++j)
+        // that its MMAs can start as soon as the accumulator is read.
+        // A single-tile CTA takes turns with the other grid's CTA on its SM
+        // (g_sm_turn): its early unpacks wait for that CTA's late ones, and
+        // it marks the SM while its own late unpacks are pending.
+        const bool turns = wk.ntiles == 1 && nst > C::A_STAGES;
+        if (turns && lane == 0) sm_turn_wait(sm_id(), grid_tag());
+        __syncwarp();
+        for (int j = pre; j < nst; ++j) {
           if (!unpack_stage()) { ok = false; break; }
+          if (turns && j == C::A_STAGES - 1 && warp == 2 && lane == 0) {
+            atomicExch(&g_sm_turn[sm_id()], grid_tag());
+            marked = true;
+          }
+        }
+        if (marked) {
+          atomicCAS(&g_sm_turn[sm_id()], grid_tag(), 0u);
+          marked = false;
+        }
         pre = 0;
         if (ok && t + 1 < wk.ntiles) {
           for (int j = 0; j < (nst < C::PREFILL ? nst : C::PREFILL); ++j, ++pre)
