@@ -11,7 +11,7 @@ def _layer(fmt="int4", K=256, N=128):
     # a layer object without a library handle: only the argument checks run
     lin = dq.QuantizedLinear.__new__(dq.QuantizedLinear)
     lin._h, lin.fmt, lin.K, lin.N, lin.act_scale = None, fmt, K, N, None
-    lin.device, lin._check_current = torch.device("cuda", 0), False
+    lin.device, lin._dev, lin._check_current = torch.device("cuda", 0), 0, False
     return lin
 
 
@@ -119,7 +119,10 @@ def test_x_on_another_device_is_rejected():
         def is_contiguous(self):
             return True
 
+        def get_device(self):
+            return 1
+
     lin = _layer()
-    assert not _fits(OnDevice1(), 256, torch.bfloat16, device=lin.device)
+    assert not _fits(OnDevice1(), 256, torch.bfloat16, dev=lin._dev)
     with pytest.raises(ValueError, match="expected cuda:0"):
         lin(OnDevice1())

@@ -54,15 +54,30 @@ def _require(t, name, shape=None, dtype=None, nbytes=None, device=None):
         raise ValueError(f"{name} must hold {nbytes} bytes, got {t.numel() * t.element_size()}")
 
 
-def _fits(t, cols, dtype, rows=None, device=None):
+def _fits(t, cols, dtype, rows=None, dev=None):
     """Fast form of the _require checks for a 2-D operand [rows, cols]: True
-    exactly when _require(t, shape=(rows, cols), dtype, device) would pass."""
+    exactly when _require(t, shape=(rows, cols), dtype, device) would pass,
+    `dev` being that device's index (an integer compare: building the
+    operand's torch.device on every call costs more than the rest)."""
     try:
         return (t.dtype is dtype and t.is_cuda and t.dim() == 2 and t.shape[1] == cols
                 and (rows is None or t.shape[0] == rows) and t.is_contiguous()
-                and (device is None or t.device == device))
+                and (dev is None or t.get_device() == dev))
     except AttributeError:
         return False
+
+
+_torch_mod = None
+
+
+def _torch():
+    """torch, imported on first use (the package itself does not need it)."""
+    global _torch_mod
+    if _torch_mod is None:
+        import torch
+
+        _torch_mod = torch
+    return _torch_mod
 
 
 def _storage_bytes(fmt, K, N):
@@ -76,18 +91,17 @@ def static_mlp(l1, l2, x, out=None, h_out=None, stream=None):
     with l2.K == l1.N, l1.N in {256, 512, 1024}, l2.N <= 128; x bf16
     [M, l1.K] on their device.  Returns y (``out``, allocated if None);
     ``h_out`` (bf16 [M, l1.N]) receives layer 1's output if given."""
-    import torch
-
+    torch = _torch()
     if l1.fmt != "fp8_static" or l2.fmt != "fp8_static":
         raise ValueError("static_mlp needs two fp8_static layers")
     if l2.K != l1.N:
         raise ValueError(f"layer 2 takes {l2.K} inputs, layer 1 gives {l1.N}")
-    if l2.device != l1.device:
+    if l2._dev != l1._dev:
         raise ValueError("both layers must live on the same device")
     M = l1._check_x(x, torch.bfloat16)
-    out = l2._out(out, M, torch.bfloat16, x.device)
+    out = l2._out(out, M, torch.bfloat16)
     if h_out is not None:
-        _require(h_out, "h_out", shape=(M, l1.N), dtype=torch.bfloat16, device=x.device)
+        _require(h_out, "h_out", shape=(M, l1.N), dtype=torch.bfloat16, device=l1.device)
     if M == 0:
         return out
     dqgemm_run_static_mlp(l1.handle, l2.handle, x, M, h_out, out, stream)
@@ -128,6 +142,7 @@ class QuantizedLinear:
         self._static_prequant_m = (self.STATIC_PREQUANT_M_WIDE if 2 * n_tiles > sms and n_tiles <= sms
                                    else self.STATIC_PREQUANT_M)
         self.device = packed.device               # the handle belongs to this device
+        self._dev = self.device.index
         # with one visible GPU the current device can only be this one
         self._check_current = torch.cuda.device_count() > 1
         self.act_scale = float(global_scale) if fmt == "fp8_static" else None
@@ -153,55 +168,50 @@ class QuantizedLinear:
         return cls(fmt, K, N, packed, scales, g, bias)
 
     def _check_x(self, x, dtype, name="x"):
-        if not _fits(x, self.K, dtype, device=self.device):
+        if not _fits(x, self.K, dtype, dev=self._dev):
             if getattr(x, "dim", lambda: 0)() != 2:
                 raise ValueError(f"{name} must be 2-D [M, {self.K}]")
             _require(x, name, shape=(x.shape[0], self.K), dtype=dtype, device=self.device)
         if self._check_current:
-            import torch
-
-            if torch.cuda.current_device() != self.device.index:
+            if _torch().cuda.current_device() != self._dev:
                 raise ValueError(f"the layer lives on {self.device}; make it the current device "
                                  f"(torch.cuda.set_device / torch.cuda.device) before calling it")
         return x.shape[0]
 
-    def _out(self, out, M, dtype, device):
+    def _out(self, out, M, dtype):
         if out is None:
-            import torch
-
-            return torch.empty((M, self.N), dtype=dtype, device=device)
-        if not _fits(out, self.N, dtype, M, device):
-            _require(out, "out", shape=(M, self.N), dtype=dtype, device=device)
+            return _torch().empty((M, self.N), dtype=dtype, device=self.device)
+        if not _fits(out, self.N, dtype, M, self._dev):
+            _require(out, "out", shape=(M, self.N), dtype=dtype, device=self.device)
         return out
 
     def __call__(self, x, out=None, stream=None):
         """y = x . deq(W)^T + b; x bf16 [M, K] contiguous on CUDA, y (``out``,
         allocated if None) bf16 [M, N]."""
-        import torch
-
+        torch = _torch()
         M = self._check_x(x, torch.bfloat16)
-        out = self._out(out, M, torch.bfloat16, x.device)
+        out = self._out(out, M, torch.bfloat16)
         if M == 0:
             return out
         if self.fmt == "fp8_static" and M >= self._static_prequant_m:
-            q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
+            q = torch.empty((M, self.K), dtype=torch.uint8, device=self.device)
             dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
             dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)
         else:
-            dqgemm_run(self._h, x, M, out, stream)
+            # (operands checked above: their pointers go straight to the entry)
+            _native.run_ptrs(self._h, x.data_ptr(), M, out.data_ptr(), stream)
         return out
 
     def quantized_out(self, x, s_out, out=None, stream=None):
         """The layer with its result leaving as the next static-FP8 layer's
         e4m3 codes, e4m3(f32(y) / s_out) (uint8 [M, N]); x as for __call__."""
-        import torch
-
+        torch = _torch()
         M = self._check_x(x, torch.bfloat16)
-        out = self._out(out, M, torch.uint8, x.device)
+        out = self._out(out, M, torch.uint8)
         if M == 0:
             return out
         if self.fmt == "fp8_static" and M >= self._static_prequant_m:
-            q = torch.empty((M, self.K), dtype=torch.uint8, device=x.device)
+            q = torch.empty((M, self.K), dtype=torch.uint8, device=self.device)
             dqgemm_quantize_act_fp8(x, M, self.K, self.act_scale, q, stream)
             dqgemm_run_fp8_static_quantized_out(self._h, q, M, out, s_out, stream)
         else:
@@ -216,7 +226,7 @@ class QuantizedLinear:
         if self.fmt != "fp8_static":
             raise ValueError("from_codes needs a static FP8 layer")
         M = self._check_x(q, torch.uint8, "q")
-        out = self._out(out, M, torch.bfloat16, q.device)
+        out = self._out(out, M, torch.bfloat16)
         if M == 0:
             return out
         dqgemm_run_fp8_static_quantized(self._h, q, M, out, stream)

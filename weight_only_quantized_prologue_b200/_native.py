@@ -130,6 +130,12 @@ def dqgemm_run(h, x, M, y, stream=None):
     _check(lib().dqgemm_run(h, _ptr(x), int(M), _ptr(y), _stream(stream)), "dqgemm_run")
 
 
+def run_ptrs(h, x_ptr, M, y_ptr, stream=None):
+    """dqgemm_run on raw device addresses, for callers that have checked the
+    operands already (QuantizedLinear's per-call path)."""
+    _check(lib().dqgemm_run(h, x_ptr, M, y_ptr, _stream(stream)), "dqgemm_run")
+
+
 def dqgemm_run_fp8_static_quantized(h, q, M, y, stream=None):
     _check(lib().dqgemm_run_fp8_static_quantized(h, _ptr(q), int(M), _ptr(y), _stream(stream)),
            "dqgemm_run_fp8_static_quantized")
