@@ -528,9 +528,10 @@ def single_launch_us(torch, sets, stream, reps=8):
 
 
 class EndToEnd:
-    """The step through the public API with its data on the host: every step
-    copies its inputs from pinned host memory (one packed copy) and its
-    results back (one packed copy).  Uploads and downloads run on streams of
+    """The step through the C ABI (its binding's dqgemm_run and
+    dqgemm_run_static_mlp) with its data on the host: every step copies its
+    inputs from pinned host memory (one packed copy) and its results back
+    (one packed copy).  Uploads and downloads run on streams of
     their own over a ring of NB buffers, so later steps' inputs go up and
     earlier steps' results come down while step i computes; every byte of
     every step still crosses, inside the timed region."""
@@ -542,6 +543,7 @@ class EndToEnd:
     def __init__(self, torch, dq, sets, stream):
         self.torch, self.dq, self.sets, self.compute = torch, dq, sets, stream
         self.up, self.down = torch.cuda.Stream(), torch.cuda.Stream()
+        self.cs = stream.cuda_stream              # the compute stream's handle, for the C calls
         s0 = sets[0]
         xs = {f: s0.x for f in LIN_FORMATS}
         xs["fp8_static_l1"] = s0.xm
@@ -595,9 +597,9 @@ class EndToEnd:
             if i >= self.NB:
                 self.compute.wait_event(self.ev["down"][b])       # step i-NB's results are home
             for f in LIN_FORMATS:
-                st.layers[f](xin[f], out=yout[f], stream=self.compute)
-            self.dq.static_mlp(st.mlp1, st.mlp2, xin["fp8_static_l1"], out=yout["fp8_static_l2"],
-                               stream=self.compute)
+                self.dq.dqgemm_run(st.layers[f].handle, xin[f], LM, yout[f], self.cs)
+            self.dq.dqgemm_run_static_mlp(st.mlp1.handle, st.mlp2.handle, xin["fp8_static_l1"], LM, None,
+                                          yout["fp8_static_l2"], self.cs)
             self.ev["done"][b].record(self.compute)
             with torch.cuda.stream(self.down):
                 self.down.wait_event(self.ev["done"][b])
