@@ -565,9 +565,11 @@ class EndToEnd:
         self.h_out = [torch.empty(n_out, dtype=bf).pin_memory() for _ in range(nb)]
         self.d_in = [torch.empty(n_in, dtype=bf, device="cuda") for _ in range(nb)]
         self.d_out = [torch.empty(n_out, dtype=bf, device="cuda") for _ in range(nb)]
-        # per-call operand views into each packed buffer, made once
-        self.vin = [dict(zip(self.IN, self._views(self.d_in[b], self.in_shapes))) for b in range(nb)]
-        self.vout = [dict(zip(self.OUT, self._views(self.d_out[b], self.out_shapes))) for b in range(nb)]
+        # per-call operand addresses in each packed buffer, taken once
+        self.vin = [{n: v.data_ptr() for n, v in zip(self.IN, self._views(self.d_in[b], self.in_shapes))}
+                    for b in range(nb)]
+        self.vout = [{n: v.data_ptr() for n, v in zip(self.OUT, self._views(self.d_out[b], self.out_shapes))}
+                     for b in range(nb)]
         self.ev = {k: [torch.cuda.Event() for _ in range(nb)] for k in ("up", "done", "down")}
 
     @staticmethod

@@ -87,8 +87,10 @@ def _check(status, what):
 
 
 def _ptr(t):
-    if t is None:
-        return None
+    """A buffer's address: a tensor's data_ptr, a NumPy array's data, or an
+    address given as an integer (the C entry points take plain pointers)."""
+    if t is None or type(t) is int:
+        return t
     if isinstance(t, np.ndarray):
         return t.ctypes.data_as(ctypes.c_void_p).value
     return t.data_ptr()
