@@ -126,3 +126,18 @@ def test_x_on_another_device_is_rejected():
     assert not _fits(OnDevice1(), 256, torch.bfloat16, dev=lin._dev)
     with pytest.raises(ValueError, match="expected cuda:0"):
         lin(OnDevice1())
+
+
+def test_buffers_may_be_given_as_integer_addresses():
+    # the C entry points take plain pointers: the binding passes an integer
+    # address through unchanged, takes a tensor's data_ptr and an array's data
+    import numpy as np
+
+    from weight_only_quantized_prologue_b200 import _native
+
+    assert _native._ptr(None) is None
+    assert _native._ptr(0x7F0000001000) == 0x7F0000001000
+    a = np.zeros(4, dtype=np.float32)
+    assert _native._ptr(a) == a.ctypes.data
+    t = torch.zeros(4)
+    assert _native._ptr(t) == t.data_ptr()
