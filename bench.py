@@ -500,11 +500,14 @@ def wide_block(torch, dq, synthetic, stream, peaks, reps=24):
     return out
 
 
-def single_launch_us(torch, sets, stream, reps=8):
-    """Median device time of one call on its own: the stream is idle apart
+def single_launch_us(torch, sets, stream, reps=32):
+    """Mean device time of one call on its own: the stream is idle apart
     from an L2 flush (a 256 MB memset) before it, so the call neither
     overlaps a neighbour nor finds its weight in L2.  Per weight-only format;
-    None if the measurement itself fails (it is outside the timed step)."""
+    None if the measurement itself fails (it is outside the timed step).
+    (The event clock ticks about once a microsecond: single intervals are
+    multiples of the tick, and a mean over many calls, whose starts fall at
+    random phases of the tick, resolves below it.)"""
     try:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
         out = {}
@@ -520,7 +523,7 @@ def single_launch_us(torch, sets, stream, reps=8):
                     z.record(stream)
                     z.synchronize()
                     lat.append(a.elapsed_time(z) * 1000.0)
-                out[f] = round(statistics.median(lat), 3)
+                out[f] = round(statistics.fmean(lat), 3)
         del flush
         return out
     except Exception as e:      # noqa: BLE001 - report, do not lose the bench line
